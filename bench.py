@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the RACE attention hot path on B200; prints one JSON line.
+
+A step is one pass of the whole hot path over one batch of synthetic input: the
+forward (soft hash, sketch build, prefix scan, readout) and the backward (dq, dk, dv,
+dW) of the causal 4M-token workload (8 heads, d = 64, L = 16, P = 8, tau = 0.25,
+chunk 256, clustered q/k) unless --workload says otherwise.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU: heads are independent, so every rank
+processes its own batch of heads (weak scaling) and the only exchange is the sum of
+dW over ranks (NCCL all-reduce), as in data-parallel training of the layer.
+Timing: CUDA events on the launching stream, barrier + synchronize on both sides,
+max over ranks.  Inputs (12.9 GB of q, k, v) are far larger than L2.
+
+--impl reference times the float64 CPU oracle (the reference arm of this repo) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_lsh_sketch_race_b200 import inputs as I  # noqa: E402
+
+METRIC = "RACE attn tokens/s (fwd, fwd+bwd) at N=4M causal; % of tensor/HBM roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+def flops_per_token_head(wl: I.Workload):
+    """Algorithmic work of the method per token and head (chunk-independent):
+    forward 4*LR*(d+1) + 4*d*L*P (state build, readout, q/k projections);
+    backward 10*LR*(d+1) + 12*d*L*P."""
+    LR = wl.L * wl.R
+    fwd = 4 * LR * (wl.d + 1) + 4 * wl.d * wl.L * wl.P
+    bwd = 10 * LR * (wl.d + 1) + 12 * wl.d * wl.L * wl.P
+    return fwd, bwd
+
+
+def bytes_per_token_head(wl: I.Workload):
+    """HBM bytes the method must move: read q, k, v, write o (forward); read q, k, v,
+    o, dO, den, write dq, dk, dv (backward)."""
+    es = 2 if wl.dtype == "bf16" else 4
+    return 4 * wl.d * es, 8 * wl.d * es + 4
+
+
+# Per-launch algorithmic flops of each kernel, as a multiple of (token-heads seen by
+# one launch).  Kernels missing here are not candidates for the roofline line.
+def kernel_work(name: str, wl: I.Workload):
+    LR, d, L, P = wl.L * wl.R, wl.d, wl.L, wl.P
+    th = wl.H * wl.N
+    table = {
+        "simt_readout_sweep": 4 * LR * (d + 1) + 4 * d * L * P if wl.causal else 2 * LR * (d + 1) + 2 * d * L * P,
+        "simt_sketch_build": 2 * LR * (d + 1) + 2 * d * L * P,
+        "simt_bwd_q": 4 * LR * (d + 1) + 8 * d * L * P,
+        "simt_bwd_kv": 6 * LR * (d + 1) + 8 * d * L * P,
+        "tc_causal_sweep": 4 * LR * (d + 1) + 4 * d * L * P,
+        "tc_sketch_build": 2 * LR * (d + 1) + 2 * d * L * P,
+        "tc_readout": 2 * LR * (d + 1) + 2 * d * L * P,
+    }
+    if name not in table:
+        return None
+    return table[name] * th
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- oracle arm
+def oracle_rate(wl: I.Workload, n_tokens: int, backward: bool, seed_head: int = 0):
+    """Time the float64 oracle on one head of n_tokens tokens; returns (tokens/s of the
+    whole multi-head workload, seconds, threads)."""
+    import numpy as np  # noqa: F401
+    import oracle
+    x = I.make_inputs(wl, "cpu", N=n_tokens, heads=[seed_head], with_dout=True)
+    f = {k: v.double().numpy() for k, v in x.items()}
+    t0 = time.perf_counter()
+    if backward:
+        oracle.backward(f["q"][0], f["k"][0], f["v"][0], f["W"], wl.tau, wl.causal,
+                        f["dout"][0])
+    else:
+        oracle.forward(f["q"][0], f["k"][0], f["v"][0], f["W"], wl.tau, wl.causal)
+    dt = time.perf_counter() - t0
+    # one head of n tokens is 1/H of the per-token work of the full workload
+    tokens_equiv = n_tokens * wl.batch / wl.H
+    return tokens_equiv / dt, dt, os.cpu_count()
+
+
+def run_reference(args, wl: I.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    backward = not args.fwd_only
+    n = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_rate(wl, n, backward)
+    times = []
+    for s in range(args.steps):
+        rate, dt, cores = oracle_rate(wl, n, backward, seed_head=s % wl.H)
+        times.append(dt)
+    ms = 1000 * statistics.mean(times)
+    value = n * wl.batch / wl.H / (ms / 1000)
+    unit = "tokens/s"
+    sample = (f"one head of {n} tokens of the {wl.name} workload per step "
+              f"({'forward+backward' if backward else 'forward'}), float64 numpy oracle; "
+              f"tokens/s scaled by 1/{wl.H} heads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "H": wl.H, "N": wl.N, "d": wl.d, "L": wl.L,
+                   "P": wl.P, "tau": wl.tau, "causal": wl.causal,
+                   "step": "fwd+bwd" if backward else "fwd"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": os.cpu_count(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_ours(args, wl: I.Workload):
+    import torch.distributed as dist
+
+    from linear_lsh_sketch_race_b200 import race_attn as ra
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+    ra.load()
+    backward = not args.fwd_only
+    heads = [rank * wl.H + h for h in range(wl.H)]
+    x = I.make_inputs(wl, dev, heads=heads, with_dout=backward)
+    q, k, v, W = x["q"], x["k"], x["v"], x["W"]
+    dout = x.get("dout")
+    out = torch.empty_like(q)
+    den = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    a = ra.make_args(q, W, wl.tau, wl.causal, chunk=wl.chunk, impl=args.kernels, den=den)
+    need = max(ra.race_workspace_size(a, False),
+               ra.race_workspace_size(a, True) if backward else 0)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    a.workspace = ws.data_ptr()
+    a.workspace_bytes = ws.numel()
+    if backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dW = torch.empty_like(W)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd_only():
+        ra.race_forward_ex(q, k, v, W, out, a, stream)
+
+    def step():
+        ra.race_forward_ex(q, k, v, W, out, a, stream)
+        if backward:
+            ra.race_backward_ex(q, k, v, W, out, dout, dq, dk, dv, dW, a, stream)
+            if world > 1:
+                dist.all_reduce(dW)
+
+    def timed(fn, n):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        ms = e0.elapsed_time(e1) / n
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = t.item()
+        return ms
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert ra.race_device_status(stream) == 0
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ra.race_timing_enable(True)
+    n0 = ra.race_launch_count()
+    ms = timed(step, args.steps)
+    launches = ra.race_launch_count() - n0
+    ktimes = ra.race_timing_report()
+    ra.race_timing_enable(False)
+    clocks = sampler.stop()
+    if ra.race_device_status(stream) != 0:
+        raise RuntimeError("device status flag raised during the timed region")
+    fwd_ms = timed(fwd_only, args.steps) if backward else ms
+
+    tokens = wl.batch * wl.N * world
+    value = tokens / (ms / 1000)
+    peaks, peak_src = load_peaks()
+    f_fwd, f_bwd = flops_per_token_head(wl)
+
+    # dominant kernel of the step, against the sustained tensor peak
+    roof = None
+    cands = [(t[0], n) for n, t in ktimes.items() if kernel_work(n, wl) is not None]
+    if cands:
+        tot, name = max(cands)
+        ms_launch = ktimes[name][0] / ktimes[name][1]
+        work = kernel_work(name, wl)
+        achieved = work / (ms_launch / 1000) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "ms_per_launch": ms_launch, "flops_per_launch": work,
+                "share_of_step": tot / sum(t[0] for t in ktimes.values())}
+
+    ideal_ms = max(wl.H * wl.N * (f_fwd + (f_bwd if backward else 0)) /
+                   (peaks["bf16_tflops"] * 1e12),
+                   wl.H * wl.N * sum(bytes_per_token_head(wl)[: 2 if backward else 1]) /
+                   (peaks["hbm_gbs"] * 1e9)) * 1000
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "H": wl.H, "N": wl.N, "d": wl.d, "L": wl.L,
+                   "P": wl.P, "tau": wl.tau, "causal": wl.causal, "chunk": wl.chunk,
+                   "step": "fwd+bwd" if backward else "fwd", "kernels": args.kernels,
+                   "l2": "inputs larger than L2 (q, k, v = %.1f GB per rank)" %
+                         (3 * q.numel() * q.element_size() / 1e9),
+                   "parallelism": f"heads sharded: {wl.H} heads per rank"},
+        "fwd": {"value": tokens / (fwd_ms / 1000), "unit": "tokens/s",
+                "ms_per_step": fwd_ms},
+        "method_roofline": {"ideal_ms_per_step": ideal_ms, "frac": ideal_ms / ms,
+                            "peak_source": f"{peak_src} bf16_tflops (burst) / hbm_gbs"},
+        "roofline": roof,
+        "kernel_ms_per_step": {n: t[0] / args.steps for n, t in ktimes.items()},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, wl, x, a, ra, dev, stream, world, backward)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_tokens
+        rate, dt, cores = oracle_rate(wl, n, backward)
+        line["cpu_baseline"] = {
+            "value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"one head of {n} tokens ({'fwd+bwd' if backward else 'fwd'}), "
+                      f"{dt:.1f} s of float64 numpy; tokens/s scaled by 1/{wl.H} heads"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, wl, x, a, ra, dev, stream, world, backward):
+    """Same step through the public API with host inputs: pinned host -> device copies
+    of q, k, v (and dO), the step, device -> host copies of the results."""
+    try:
+        import torch.distributed as dist
+        names = ["q", "k", "v"] + (["dout"] if backward else [])
+        host = {n: torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True) for n in names}
+        for n in names:
+            host[n].copy_(x[n])
+        dev_in = {n: torch.empty_like(x[n]) for n in names}
+        W = x["W"]
+        out = torch.empty_like(x["q"])
+        outs = [out]
+        if backward:
+            grads = [torch.empty_like(x["q"]), torch.empty_like(x["k"]),
+                     torch.empty_like(x["v"]), torch.empty_like(W)]
+            outs += grads
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+
+        def step():
+            for n in names:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            ra.race_forward_ex(dev_in["q"], dev_in["k"], dev_in["v"], W, out, a, stream)
+            if backward:
+                ra.race_backward_ex(dev_in["q"], dev_in["k"], dev_in["v"], W, out,
+                                    dev_in["dout"], *grads, a, stream)
+                if world > 1:
+                    dist.all_reduce(grads[3])
+            for t, h in zip(outs, host_out):
+                h.copy_(t, non_blocking=True)
+
+        n = max(1, min(args.steps, args.e2e_steps))
+        step()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / n
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = t.item()
+        tokens = wl.batch * wl.N * world
+        return {"value": tokens / (ms / 1000), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms, "steps": n}
+    except Exception as e:  # pinned host memory can be short on some hosts
+        return {"value": None, "unit": "tokens/s", "error": repr(e)[:200]}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=I.HEADLINE, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--N", type=int, default=0, help="override sequence length")
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--kernels", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=8192)
+    ap.add_argument("--ref-tokens", type=int, default=2048)
+    args = ap.parse_args()
+    wl = I.WORKLOADS[args.workload]
+    if args.N:
+        wl = wl.replace(N=args.N, name=f"{wl.name}_N{args.N}")
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+/*
+ * race_attn.h — C ABI of the RACE attention library (librace_attn.so).
+ *
+ * RACE attention estimates attention under the sharpened angular kernel
+ *     sim(q, k) = (1 - arccos(qhat . khat) / pi)^P
+ * with L repeated arrays of P-bit signed-random-projection buckets (R = 2^P) and
+ * soft hashing.  Sources, by page title:
+ *   [JA]  "RACE Attention: 長系列トレーニングのための厳密な線形時間アテンションの技術的概要"
+ *         (gist.science, Japanese technical overview), §2.1 core idea (sim equation,
+ *         soft bucketization, bucket aggregation, reconstruction), §2.2 (differentiable
+ *         soft assignment with temperature; prefix-sum kernels for causal masking;
+ *         complexity O(L N R d)).
+ *   [IT]  "RACE Attention: A Strictly Linear-Time Attention for Long-Sequence
+ *         Training" (gist.science, Italian technical summary), §2 (random projections
+ *         softened by a softmax over the hypercube vertices; per-bucket mass and value
+ *         sums; normalised weighted mean), §3 (causal and non-causal kernels).
+ *   [ABS] "Replacing Softmax Similarity with a Sharpened Angular Similarity ..."
+ *         (arXiv 2510.04008 abstract): forward-backward of a multi-head attention layer.
+ *
+ * The operation, fixed exactly:
+ *     xhat = x / max(|x|_2, 1e-12)
+ *     u_l  = W_l^T xhat                         (W: [L, d, P], plane p of table l = W[l,:,p])
+ *     p_l  = softmax_b(<c_b, u_l> / tau)        (b = 0..R-1, c_bp = +1 iff bit p of b is set)
+ *     phi  = concat_l p_l / sqrt(L)             ([L*R] per vector)
+ *     o_i  = sum_{j in J(i)} (phi(q_i).phi(k_j)) v_j / sum_{j in J(i)} phi(q_i).phi(k_j)
+ *     J(i) = all j (non-causal) or j <= i (causal, inclusive).
+ *
+ * Layouts.  q, k, v, out, dout, dq, dk, dv are dense row-major [H][N][d] with
+ * H = batch * heads (W is shared by every head).  W and dW are dense [L][d][P]
+ * float32.  den is [H][N] float32.  phi dumps are [H][N][L*R].
+ *
+ * Pointers.  Every tensor pointer is a DEVICE pointer on the current CUDA device,
+ * except where an entry point says "host".  Tensor pointers must be 16-byte aligned.
+ * The caller owns every buffer; the library keeps no pointer after a call returns.
+ *
+ * Execution.  Calls enqueue work on `stream` and return without synchronising
+ * (cudaStream_t; NULL is the legacy default stream).  They never print, abort or
+ * exit.  Argument errors are reported before anything is enqueued.
+ *
+ * Supported sizes: d = 64; 1 <= P <= 8; L >= 1 with L * 2^P <= 16384; N >= 1;
+ * H >= 1; tau finite and > 0.  Other d values give RACE_ERR_UNSUPPORTED.
+ */
+#ifndef RACE_ATTN_H
+#define RACE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *race_stream_t;
+
+typedef enum {
+  RACE_OK = 0,
+  RACE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad tau          */
+  RACE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d != 64)             */
+  RACE_ERR_WORKSPACE = 3,     /* caller workspace too small or allocation failed     */
+  RACE_ERR_CUDA = 4,          /* a CUDA runtime call or a launch failed              */
+  RACE_ERR_DEVICE_STATUS = 5  /* a kernel raised its device status flag (a bounded   */
+                              /* wait gave up, or an index check failed)             */
+} race_status_t;
+
+typedef enum { RACE_BF16 = 0, RACE_FP32 = 1 } race_dtype_t;
+
+/* Which kernels a call may use.  AUTO picks the tensor-core (tcgen05) path for
+ * bf16 inputs where it exists and the CUDA-core path otherwise.  SIMT forces the
+ * CUDA-core kernels (always available; the only path for fp32).  TENSOR forces the
+ * tensor-core kernels and fails with RACE_ERR_UNSUPPORTED where they do not apply. */
+typedef enum { RACE_IMPL_AUTO = 0, RACE_IMPL_SIMT = 1, RACE_IMPL_TENSOR = 2 } race_impl_t;
+
+/* Full argument set of the *_ex entry points. */
+typedef struct {
+  int64_t N;                 /* sequence length                                        */
+  int H;                     /* batch * heads                                          */
+  int d;                     /* head dimension (64)                                    */
+  int L;                     /* number of hash tables                                  */
+  int P;                     /* hyperplanes per table; R = 2^P buckets                 */
+  float tau;                 /* soft-hash temperature (the pages' beta is 1/tau)       */
+  int causal;                /* 0: all keys; 1: keys j <= i                            */
+  race_dtype_t dtype;        /* element type of q, k, v, dout, dq, dk, dv              */
+  race_dtype_t out_dtype;    /* element type of out (forward writes, backward reads)   */
+  int chunk;                 /* tokens per chunk of the causal sweep; 0 = library      */
+                             /* choice; otherwise a multiple of 64 (tensor-core path)   */
+                             /* or of 32 (CUDA-core path)                               */
+  void *workspace;           /* device scratch of >= workspace_bytes, or NULL: the      */
+  size_t workspace_bytes;    /* library then allocates stream-ordered scratch itself    */
+  float *den;                /* optional [H][N]: forward writes den_i =                 */
+                             /* sum_j phi(q_i).phi(k_j); backward reads it (NULL: the   */
+                             /* backward recomputes it)                                 */
+  race_impl_t impl;          /* kernel family, see race_impl_t                          */
+} race_args_t;
+
+/* Fill `a` with the defaults of the spec-form calls: bf16 in and out, chunk 0,
+ * no workspace, no den, RACE_IMPL_AUTO. */
+void race_args_init(race_args_t *a, int64_t N, int H, int d, int L, int P, float tau,
+                    int causal);
+
+/* ---------------------------------------------------------------------------------
+ * race_forward — RACE attention forward, bf16 q/k/v/out, float32 W.
+ * Soft hash, bucket aggregation (S = sum phi(k) v^T, z = sum phi(k)), readout and
+ * normalisation: [JA] §2.1 (soft bucketization, bucket aggregation, reconstruction),
+ * causal prefix sums: [JA] §2.2.  Allocates stream-ordered scratch on `stream`
+ * (cudaMallocAsync / cudaFreeAsync).
+ * Returns RACE_OK, RACE_ERR_INVALID_ARG, RACE_ERR_UNSUPPORTED, RACE_ERR_WORKSPACE or
+ * RACE_ERR_CUDA.
+ * ------------------------------------------------------------------------------ */
+race_status_t race_forward(const void *q, const void *k, const void *v, const float *W,
+                           void *out, int64_t N, int H, int d, int L, int P, float tau,
+                           int causal, race_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * race_backward — gradients of sum(out * dout) with respect to q, k, v and W
+ * (differentiable soft assignment, [JA] §2.2 and [IT] §3 item 4; the formulas are the
+ * chain rule of the forward).  bf16 q/k/v/out/dout/dq/dk/dv; dW float32, OVERWRITTEN
+ * with the sum over all heads and tokens.  `out` must be the forward's output for the
+ * same inputs.  den is recomputed.  Scratch as in race_forward.
+ * ------------------------------------------------------------------------------ */
+race_status_t race_backward(const void *q, const void *k, const void *v, const float *W,
+                            const void *out, const void *dout, void *dq, void *dk,
+                            void *dv, float *dW, int64_t N, int H, int d, int L, int P,
+                            float tau, int causal, race_stream_t stream);
+
+/* Extended forms: every option in `a` (dtypes, chunk, caller workspace, den, impl). */
+race_status_t race_forward_ex(const void *q, const void *k, const void *v, const float *W,
+                              void *out, const race_args_t *a, race_stream_t stream);
+race_status_t race_backward_ex(const void *q, const void *k, const void *v,
+                               const float *W, const void *out, const void *dout,
+                               void *dq, void *dk, void *dv, float *dW,
+                               const race_args_t *a, race_stream_t stream);
+
+/* Scratch bytes the *_ex calls need for `a` (backward != 0: the backward).  Writes 0
+ * and returns an error status for invalid or unsupported arguments.  Host only; no
+ * device work. */
+race_status_t race_workspace_size(const race_args_t *a, int backward, size_t *bytes);
+
+/* ---------------------------------------------------------------------------------
+ * race_hash — the feature map alone: L2 normalisation, the d x (L*P) projection and
+ * the softmax over the 2^P corners, phi = concat_l p_l / sqrt(L) ([JA] §2.1 soft
+ * bucketization; [IT] §2 item 2).  x: [H][N][d] of a->dtype; phi: [H][N][L*2^P] of
+ * a->out_dtype (bf16 or float32).  Uses a->N, H, d, L, P, tau only.  Writes
+ * H*N*L*2^P elements: meant for checks and small problems.
+ * ------------------------------------------------------------------------------ */
+race_status_t race_hash(const void *x, const float *W, void *phi, const race_args_t *a,
+                        race_stream_t stream);
+
+/* Synchronises `stream`, then reports and clears this device's status flag, which a
+ * kernel raises when a bounded wait gives up or an index check fails.  *flags (may be
+ * NULL) receives the raw flag bits.  Returns RACE_OK or RACE_ERR_DEVICE_STATUS (or
+ * RACE_ERR_CUDA). */
+race_status_t race_device_status(race_stream_t stream, uint32_t *flags);
+
+/* Static description of a status code. */
+const char *race_status_string(race_status_t s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int race_version(void);
+
+/* ---------------------------------------------------------------------------------
+ * Profiling aids (host only).
+ * race_timing_enable(1) clears the per-kernel totals and makes every later kernel
+ * launch of the library record a CUDA event before and after it on its own stream;
+ * race_timing_enable(0) stops recording.  race_timing_report(i, ...) gives the i-th
+ * kernel seen while recording was on: its name (valid until the next
+ * race_timing_enable), the summed device time in milliseconds and the number of
+ * launches; it waits for the recorded events.  It returns RACE_ERR_INVALID_ARG once i
+ * is past the last kernel.  race_launch_count() is the number of kernel launches the
+ * library has issued in this process.
+ * ------------------------------------------------------------------------------ */
+race_status_t race_timing_enable(int on);
+race_status_t race_timing_report(int i, const char **name, double *total_ms,
+                                 int64_t *launches);
+int64_t race_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RACE_ATTN_H */

@@ -1,0 +1,575 @@
+// C-ABI implementation of librace_attn.so: argument checks, planning, scratch
+// layout and kernel launches.  The whole library is one translation unit so that the
+// device status flag is a single __device__ symbol.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "simt_kernels.cuh"
+#include "tc_kernels.cuh"
+
+namespace race {
+
+// ------------------------------------------------------------------ launch accounting
+// Every kernel launch of the library goes through a LaunchScope: it counts launches
+// and, while timing is enabled, brackets the launch with CUDA events on its stream.
+namespace launches {
+
+std::atomic<int64_t> g_count{0};
+std::mutex g_mu;
+bool g_timing = false;
+struct Timer {
+  std::string name;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending;
+  double ms = 0.0;
+  int64_t n = 0;
+};
+std::vector<Timer> g_timers;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+Timer& timer(const char* name) {
+  for (auto& t : g_timers)
+    if (t.name == name) return t;
+  g_timers.push_back(Timer{name, {}, 0.0, 0});
+  return g_timers.back();
+}
+
+// Resolve pending events into totals (synchronises on them).
+void drain() {
+  for (auto& t : g_timers) {
+    for (auto& pr : t.pending) {
+      float ms = 0.f;
+      if (cudaEventSynchronize(pr.second) == cudaSuccess &&
+          cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess) {
+        t.ms += ms;
+        t.n += 1;
+      }
+      g_pool.push_back(pr.first);
+      g_pool.push_back(pr.second);
+    }
+    t.pending.clear();
+  }
+}
+
+class Scope {
+ public:
+  Scope(const char* name, cudaStream_t s) : name_(name), s_(s) {
+    g_count.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_timing) {
+      start_ = take_event();
+      stop_ = take_event();
+      if (start_ && stop_) cudaEventRecord(start_, s_);
+    }
+  }
+  ~Scope() {
+    if (!start_ || !stop_) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaEventRecord(stop_, s_);
+    timer(name_).pending.emplace_back(start_, stop_);
+  }
+
+ private:
+  const char* name_;
+  cudaStream_t s_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
+
+}  // namespace launches
+
+#define RACE_LAUNCH(name, stream) launches::Scope race_scope_(name, stream)
+
+namespace {
+
+constexpr int kPlanSMs = 148;        // planning constant: SM count of a B200
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+race_status_t check_args(const race_args_t* a) {
+  if (!a) return RACE_ERR_INVALID_ARG;
+  if (a->N < 1 || a->H < 1 || a->L < 1 || a->d < 1) return RACE_ERR_INVALID_ARG;
+  if (a->P < 1 || a->P > 8) return RACE_ERR_INVALID_ARG;
+  if ((int64_t)a->L * (1 << a->P) > 16384) return RACE_ERR_INVALID_ARG;
+  if (!std::isfinite(a->tau) || !(a->tau > 0.f)) return RACE_ERR_INVALID_ARG;
+  if (a->causal != 0 && a->causal != 1) return RACE_ERR_INVALID_ARG;
+  if ((a->dtype != RACE_BF16 && a->dtype != RACE_FP32) ||
+      (a->out_dtype != RACE_BF16 && a->out_dtype != RACE_FP32))
+    return RACE_ERR_INVALID_ARG;
+  if (a->impl != RACE_IMPL_AUTO && a->impl != RACE_IMPL_SIMT && a->impl != RACE_IMPL_TENSOR)
+    return RACE_ERR_INVALID_ARG;
+  if (a->chunk < 0) return RACE_ERR_INVALID_ARG;
+  if ((double)a->N * a->H * a->d > 4.0e18) return RACE_ERR_INVALID_ARG;
+  if (a->d != kD) return RACE_ERR_UNSUPPORTED;
+  return RACE_OK;
+}
+
+Dims dims_of(const race_args_t* a) {
+  Dims dm;
+  dm.N = a->N;
+  dm.H = a->H;
+  dm.L = a->L;
+  dm.P = a->P;
+  dm.R = 1 << a->P;
+  dm.tau = a->tau;
+  dm.causal = a->causal;
+  return dm;
+}
+
+// ----------------------------------------------------------------------------- SIMT
+struct SimtPlan {
+  Dims dm;
+  int G;
+  int64_t seg_len;
+  size_t off_seg, off_init, off_num, off_gpp, off_dxq, off_dxk, off_dv, off_dwq, off_dwk;
+  size_t bytes;
+};
+
+SimtPlan simt_plan(const race_args_t* a, bool backward) {
+  SimtPlan p;
+  p.dm = dims_of(a);
+  const int64_t tiles = (a->N + simt::TT - 1) / simt::TT;
+  int64_t G = (2 * kPlanSMs + (int64_t)a->H * a->L - 1) / ((int64_t)a->H * a->L);
+  G = std::max<int64_t>(1, std::min<int64_t>(G, tiles));
+  int64_t seg_tiles = (tiles + G - 1) / G;
+  p.seg_len = seg_tiles * simt::TT;
+  p.G = (int)((a->N + p.seg_len - 1) / p.seg_len);
+  const size_t HN = (size_t)a->H * a->N;
+  const size_t st = (size_t)a->H * a->L * p.G * p.dm.R * kDV * sizeof(float);
+  size_t o = 0;
+  p.off_seg = o;  o = align_up(o + st);
+  p.off_init = o; o = align_up(o + st);
+  p.off_num = o;  o = align_up(o + HN * kNumStride * sizeof(float));
+  p.off_gpp = p.off_dxq = p.off_dxk = p.off_dv = p.off_dwq = p.off_dwk = o;
+  if (backward) {
+    const size_t dwp = (size_t)a->H * a->L * p.G * kD * a->P * sizeof(float);
+    p.off_gpp = o; o = align_up(o + HN * kNumStride * sizeof(float));
+    p.off_dxq = o; o = align_up(o + HN * kD * sizeof(float));
+    p.off_dxk = o; o = align_up(o + HN * kD * sizeof(float));
+    p.off_dv = o;  o = align_up(o + HN * kD * sizeof(float));
+    p.off_dwq = o; o = align_up(o + dwp);
+    p.off_dwk = o; o = align_up(o + dwp);
+  }
+  p.bytes = o;
+  return p;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)bytes);
+}
+
+#define RACE_CU(x)                              \
+  do {                                          \
+    cudaError_t e_ = (x);                       \
+    if (e_ != cudaSuccess) return RACE_ERR_CUDA; \
+  } while (0)
+
+// Segment sums and their scan for one side of the sketch (k with [v|1], or q with g'').
+template <typename T, int MODE>
+race_status_t simt_states(const SimtPlan& p, const T* x, const T* v, const float* gpp,
+                          const float* W, char* ws, int scan_mode, cudaStream_t s) {
+  const Dims& dm = p.dm;
+  simt::Layout ly(dm.R, dm.P);
+  float* seg = reinterpret_cast<float*>(ws + p.off_seg);
+  float* init = reinterpret_cast<float*>(ws + p.off_init);
+  RACE_CU(set_smem(simt::k_build<T, MODE>, ly.bytes()));
+  {
+    RACE_LAUNCH("simt_sketch_build", s);
+    simt::k_build<T, MODE><<<dim3(p.G, dm.L, dm.H), simt::NT, ly.bytes(), s>>>(
+        x, v, gpp, W, seg, dm, p.G, p.seg_len);
+  }
+  RACE_CU(cudaGetLastError());
+  const int RD = dm.R * kDV;
+  {
+    RACE_LAUNCH("simt_chunk_scan", s);
+    simt::k_scan<<<dim3((RD + 255) / 256, dm.H * dm.L), 256, 0, s>>>(seg, init, RD, p.G,
+                                                                       scan_mode);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+template <typename T>
+race_status_t simt_forward_num(const SimtPlan& p, const T* q, const T* k, const T* v,
+                               const float* W, char* ws, cudaStream_t s) {
+  const Dims& dm = p.dm;
+  int have_init = 0;
+  if (!dm.causal || p.G > 1) {
+    race_status_t st =
+        simt_states<T, 0>(p, k, v, nullptr, W, ws, dm.causal ? 0 : 2, s);
+    if (st != RACE_OK) return st;
+    have_init = 1;
+  }
+  float* num = reinterpret_cast<float*>(ws + p.off_num);
+  RACE_CU(cudaMemsetAsync(num, 0, (size_t)dm.H * dm.N * kNumStride * sizeof(float), s));
+  simt::Layout ly(dm.R, dm.P);
+  RACE_CU(set_smem(simt::k_fwd_sweep<T>, ly.bytes()));
+  {
+    RACE_LAUNCH("simt_readout_sweep", s);
+    simt::k_fwd_sweep<T><<<dim3(p.G, dm.L, dm.H), simt::NT, ly.bytes(), s>>>(
+        q, k, v, W, reinterpret_cast<float*>(ws + p.off_init), num, dm, p.G, p.seg_len,
+        have_init);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+template <typename T, typename TO>
+race_status_t simt_forward(const race_args_t* a, const T* q, const T* k, const T* v,
+                           const float* W, TO* out, char* ws, cudaStream_t s) {
+  SimtPlan p = simt_plan(a, false);
+  race_status_t st = simt_forward_num<T>(p, q, k, v, W, ws, s);
+  if (st != RACE_OK) return st;
+  const int64_t rows = (int64_t)a->H * a->N;
+  {
+    RACE_LAUNCH("simt_normalize", s);
+    simt::k_normalize<TO><<<(unsigned)((rows + 3) / 4), 256, 0, s>>>(
+        reinterpret_cast<float*>(ws + p.off_num), out, a->den, rows, 1.f / a->L);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+template <typename T, typename TO>
+race_status_t simt_backward(const race_args_t* a, const T* q, const T* k, const T* v,
+                            const float* W, const TO* out, const T* dout, T* dq, T* dk,
+                            T* dv, float* dW, char* ws, cudaStream_t s) {
+  SimtPlan p = simt_plan(a, true);
+  const Dims& dm = p.dm;
+  const int64_t rows = (int64_t)a->H * a->N;
+  simt::Layout ly(dm.R, dm.P);
+  // k-side states (prefix or total), shared by the den recompute and the q sweep
+  int have_k = 0;
+  if (!dm.causal || p.G > 1) {
+    race_status_t st = simt_states<T, 0>(p, k, v, nullptr, W, ws, dm.causal ? 0 : 2, s);
+    if (st != RACE_OK) return st;
+    have_k = 1;
+  }
+  float* num = reinterpret_cast<float*>(ws + p.off_num);
+  if (!a->den) {
+    RACE_CU(cudaMemsetAsync(num, 0, (size_t)rows * kNumStride * sizeof(float), s));
+    RACE_CU(set_smem(simt::k_fwd_sweep<T>, ly.bytes()));
+    {
+      RACE_LAUNCH("simt_readout_sweep", s);
+      simt::k_fwd_sweep<T><<<dim3(p.G, dm.L, dm.H), simt::NT, ly.bytes(), s>>>(
+          q, k, v, W, reinterpret_cast<float*>(ws + p.off_init), num, dm, p.G, p.seg_len,
+          have_k);
+    }
+    RACE_CU(cudaGetLastError());
+  }
+  float* gpp = reinterpret_cast<float*>(ws + p.off_gpp);
+  {
+    RACE_LAUNCH("simt_bwd_prep", s);
+    simt::k_gpp<T, TO><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(dout, out, num, a->den,
+                                                                   gpp, rows, (float)a->L);
+  }
+  RACE_CU(cudaGetLastError());
+  float* dxq = reinterpret_cast<float*>(ws + p.off_dxq);
+  float* dxk = reinterpret_cast<float*>(ws + p.off_dxk);
+  float* dva = reinterpret_cast<float*>(ws + p.off_dv);
+  RACE_CU(cudaMemsetAsync(dxq, 0, (size_t)rows * kD * sizeof(float), s));
+  RACE_CU(cudaMemsetAsync(dxk, 0, (size_t)rows * kD * sizeof(float), s));
+  RACE_CU(cudaMemsetAsync(dva, 0, (size_t)rows * kD * sizeof(float), s));
+  float* dwq = reinterpret_cast<float*>(ws + p.off_dwq);
+  float* dwk = reinterpret_cast<float*>(ws + p.off_dwk);
+  RACE_CU(set_smem(simt::k_bwd_q<T>, ly.bytes()));
+  {
+    RACE_LAUNCH("simt_bwd_q", s);
+    simt::k_bwd_q<T><<<dim3(p.G, dm.L, dm.H), simt::NT, ly.bytes(), s>>>(
+        q, k, v, W, reinterpret_cast<float*>(ws + p.off_init), gpp, dxq, dwq, dm, p.G,
+        p.seg_len, have_k);
+  }
+  RACE_CU(cudaGetLastError());
+  int have_q = 0;
+  if (!dm.causal || p.G > 1) {
+    race_status_t st = simt_states<T, 1>(p, q, v, gpp, W, ws, dm.causal ? 1 : 2, s);
+    if (st != RACE_OK) return st;
+    have_q = 1;
+  }
+  RACE_CU(set_smem(simt::k_bwd_kv<T>, ly.bytes()));
+  {
+    RACE_LAUNCH("simt_bwd_kv", s);
+    simt::k_bwd_kv<T><<<dim3(p.G, dm.L, dm.H), simt::NT, ly.bytes(), s>>>(
+        q, k, v, W, reinterpret_cast<float*>(ws + p.off_init), gpp, dxk, dva, dwk, dm, p.G,
+        p.seg_len, have_q);
+  }
+  RACE_CU(cudaGetLastError());
+  {
+    RACE_LAUNCH("simt_bwd_finalize_dx", s);
+    simt::k_finalize_dx<T><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(q, dxq, dq, rows);
+  }
+  {
+    RACE_LAUNCH("simt_bwd_finalize_dx", s);
+    simt::k_finalize_dx<T><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(k, dxk, dk, rows);
+  }
+  {
+    RACE_LAUNCH("simt_bwd_convert_dv", s);
+    simt::k_convert<T><<<1184, 256, 0, s>>>(dva, dv, rows * kD);
+  }
+  const int nW = a->L * kD * a->P;
+  {
+    RACE_LAUNCH("simt_dW_reduce", s);
+    simt::k_dw_reduce<<<(nW + 255) / 256, 256, 0, s>>>(dwq, dwk, dW, a->H, a->L, p.G, a->P);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+bool use_tensor_path(const race_args_t* a) {
+  if (a->impl == RACE_IMPL_SIMT) return false;
+  if (a->dtype != RACE_BF16) return false;
+  return tc::supported(a);
+}
+
+size_t workspace_bytes(const race_args_t* a, bool backward) {
+  if (!backward && use_tensor_path(a)) return tc::forward_workspace(a);
+  return simt_plan(a, backward).bytes;
+}
+
+// Scratch: the caller's, or stream-ordered memory of our own.
+struct Scratch {
+  char* ptr = nullptr;
+  bool owned = false;
+  cudaStream_t s = nullptr;
+  race_status_t acquire(const race_args_t* a, size_t need, cudaStream_t st) {
+    s = st;
+    if (need == 0) return RACE_OK;
+    if (a->workspace) {
+      if (a->workspace_bytes < need) return RACE_ERR_WORKSPACE;
+      if ((reinterpret_cast<uintptr_t>(a->workspace) & (kAlign - 1)) != 0)
+        return RACE_ERR_INVALID_ARG;
+      ptr = static_cast<char*>(a->workspace);
+      return RACE_OK;
+    }
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, need, st) != cudaSuccess) {
+      cudaGetLastError();
+      return RACE_ERR_WORKSPACE;
+    }
+    ptr = static_cast<char*>(p);
+    owned = true;
+    return RACE_OK;
+  }
+  ~Scratch() {
+    if (owned) cudaFreeAsync(ptr, s);
+  }
+};
+
+race_status_t forward_impl(const void* q, const void* k, const void* v, const float* W,
+                           void* out, const race_args_t* a, cudaStream_t s) {
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  if (!q || !k || !v || !W || !out) return RACE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W) || !aligned16(out) ||
+      (a->den && !aligned16(a->den)))
+    return RACE_ERR_INVALID_ARG;
+  const bool tensor = use_tensor_path(a);
+  if (a->impl == RACE_IMPL_TENSOR && !tensor) return RACE_ERR_UNSUPPORTED;
+  Scratch sc;
+  st = sc.acquire(a, workspace_bytes(a, false), s);
+  if (st != RACE_OK) return st;
+  if (tensor) return tc::forward(a, q, k, v, W, out, sc.ptr, s);
+  if (a->dtype == RACE_BF16) {
+    auto* qq = static_cast<const __nv_bfloat16*>(q);
+    auto* kk = static_cast<const __nv_bfloat16*>(k);
+    auto* vv = static_cast<const __nv_bfloat16*>(v);
+    if (a->out_dtype == RACE_BF16)
+      return simt_forward(a, qq, kk, vv, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s);
+    return simt_forward(a, qq, kk, vv, W, static_cast<float*>(out), sc.ptr, s);
+  }
+  auto* qq = static_cast<const float*>(q);
+  auto* kk = static_cast<const float*>(k);
+  auto* vv = static_cast<const float*>(v);
+  if (a->out_dtype == RACE_BF16)
+    return simt_forward(a, qq, kk, vv, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s);
+  return simt_forward(a, qq, kk, vv, W, static_cast<float*>(out), sc.ptr, s);
+}
+
+race_status_t backward_impl(const void* q, const void* k, const void* v, const float* W,
+                            const void* out, const void* dout, void* dq, void* dk, void* dv,
+                            float* dW, const race_args_t* a, cudaStream_t s) {
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  const void* ptrs[] = {q, k, v, W, out, dout, dq, dk, dv, dW};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return RACE_ERR_INVALID_ARG;
+  if (a->den && !aligned16(a->den)) return RACE_ERR_INVALID_ARG;
+  if (a->impl == RACE_IMPL_TENSOR) return RACE_ERR_UNSUPPORTED;
+  Scratch sc;
+  st = sc.acquire(a, workspace_bytes(a, true), s);
+  if (st != RACE_OK) return st;
+#define RACE_BWD(T, TO)                                                                  \
+  return simt_backward<T, TO>(a, static_cast<const T*>(q), static_cast<const T*>(k),     \
+                              static_cast<const T*>(v), W, static_cast<const TO*>(out),  \
+                              static_cast<const T*>(dout), static_cast<T*>(dq),          \
+                              static_cast<T*>(dk), static_cast<T*>(dv), dW, sc.ptr, s)
+  if (a->dtype == RACE_BF16) {
+    if (a->out_dtype == RACE_BF16) RACE_BWD(__nv_bfloat16, __nv_bfloat16);
+    RACE_BWD(__nv_bfloat16, float);
+  }
+  if (a->out_dtype == RACE_BF16) RACE_BWD(float, __nv_bfloat16);
+  RACE_BWD(float, float);
+#undef RACE_BWD
+}
+
+}  // namespace
+}  // namespace race
+
+using namespace race;
+
+extern "C" {
+
+void race_args_init(race_args_t* a, int64_t N, int H, int d, int L, int P, float tau,
+                    int causal) {
+  if (!a) return;
+  std::memset(a, 0, sizeof(*a));
+  a->N = N;
+  a->H = H;
+  a->d = d;
+  a->L = L;
+  a->P = P;
+  a->tau = tau;
+  a->causal = causal;
+  a->dtype = RACE_BF16;
+  a->out_dtype = RACE_BF16;
+  a->impl = RACE_IMPL_AUTO;
+}
+
+race_status_t race_forward(const void* q, const void* k, const void* v, const float* W,
+                           void* out, int64_t N, int H, int d, int L, int P, float tau,
+                           int causal, race_stream_t stream) {
+  race_args_t a;
+  race_args_init(&a, N, H, d, L, P, tau, causal);
+  return forward_impl(q, k, v, W, out, &a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+race_status_t race_backward(const void* q, const void* k, const void* v, const float* W,
+                            const void* out, const void* dout, void* dq, void* dk,
+                            void* dv, float* dW, int64_t N, int H, int d, int L, int P,
+                            float tau, int causal, race_stream_t stream) {
+  race_args_t a;
+  race_args_init(&a, N, H, d, L, P, tau, causal);
+  return backward_impl(q, k, v, W, out, dout, dq, dk, dv, dW, &a,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+race_status_t race_forward_ex(const void* q, const void* k, const void* v, const float* W,
+                              void* out, const race_args_t* a, race_stream_t stream) {
+  return forward_impl(q, k, v, W, out, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+race_status_t race_backward_ex(const void* q, const void* k, const void* v,
+                               const float* W, const void* out, const void* dout, void* dq,
+                               void* dk, void* dv, float* dW, const race_args_t* a,
+                               race_stream_t stream) {
+  return backward_impl(q, k, v, W, out, dout, dq, dk, dv, dW, a,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+race_status_t race_workspace_size(const race_args_t* a, int backward, size_t* bytes) {
+  if (bytes) *bytes = 0;
+  if (!bytes) return RACE_ERR_INVALID_ARG;
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  if (a->impl == RACE_IMPL_TENSOR && (backward || !use_tensor_path(a)))
+    return RACE_ERR_UNSUPPORTED;
+  *bytes = workspace_bytes(a, backward != 0);
+  return RACE_OK;
+}
+
+race_status_t race_hash(const void* x, const float* W, void* phi, const race_args_t* a,
+                        race_stream_t stream) {
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  if (!x || !W || !phi || !aligned16(x) || !aligned16(W) || !aligned16(phi))
+    return RACE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Dims dm = dims_of(a);
+  simt::Layout ly(dm.R, dm.P);
+  dim3 grid((unsigned)((a->N + simt::TT - 1) / simt::TT), a->H);
+#define RACE_HASH(T, TO)                                                            \
+  do {                                                                              \
+    RACE_CU(set_smem(simt::k_hash<T, TO>, ly.bytes()));                             \
+    RACE_LAUNCH("simt_hash", s);                                                    \
+    simt::k_hash<T, TO><<<grid, simt::NT, ly.bytes(), s>>>(                         \
+        static_cast<const T*>(x), W, static_cast<TO*>(phi), dm);                    \
+  } while (0)
+  if (a->dtype == RACE_BF16) {
+    if (a->out_dtype == RACE_BF16) RACE_HASH(__nv_bfloat16, __nv_bfloat16);
+    else RACE_HASH(__nv_bfloat16, float);
+  } else {
+    if (a->out_dtype == RACE_BF16) RACE_HASH(float, __nv_bfloat16);
+    else RACE_HASH(float, float);
+  }
+#undef RACE_HASH
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+race_status_t race_device_status(race_stream_t stream, uint32_t* flags) {
+  if (flags) *flags = 0;
+  RACE_CU(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  uint32_t v = 0, zero = 0;
+  RACE_CU(cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)));
+  RACE_CU(cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)));
+  if (flags) *flags = v;
+  return v ? RACE_ERR_DEVICE_STATUS : RACE_OK;
+}
+
+const char* race_status_string(race_status_t s) {
+  switch (s) {
+    case RACE_OK: return "RACE_OK";
+    case RACE_ERR_INVALID_ARG: return "RACE_ERR_INVALID_ARG: invalid argument";
+    case RACE_ERR_UNSUPPORTED: return "RACE_ERR_UNSUPPORTED: unsupported configuration";
+    case RACE_ERR_WORKSPACE: return "RACE_ERR_WORKSPACE: scratch too small or allocation failed";
+    case RACE_ERR_CUDA: return "RACE_ERR_CUDA: CUDA call or launch failed";
+    case RACE_ERR_DEVICE_STATUS: return "RACE_ERR_DEVICE_STATUS: a kernel raised the device status flag";
+  }
+  return "unknown race_status_t";
+}
+
+int race_version(void) { return 100; }
+
+race_status_t race_timing_enable(int on) {
+  std::lock_guard<std::mutex> lk(launches::g_mu);
+  launches::drain();
+  launches::g_timers.clear();
+  launches::g_timing = on != 0;
+  return RACE_OK;
+}
+
+race_status_t race_timing_report(int i, const char** name, double* total_ms,
+                                 int64_t* count) {
+  std::lock_guard<std::mutex> lk(launches::g_mu);
+  launches::drain();
+  if (i < 0 || i >= (int)launches::g_timers.size()) return RACE_ERR_INVALID_ARG;
+  const auto& t = launches::g_timers[i];
+  if (name) *name = t.name.c_str();
+  if (total_ms) *total_ms = t.ms;
+  if (count) *count = t.n;
+  return RACE_OK;
+}
+
+int64_t race_launch_count(void) { return launches::g_count.load(); }
+
+}  // extern "C"
