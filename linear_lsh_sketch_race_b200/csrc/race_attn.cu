@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace race {
 
@@ -346,6 +347,78 @@ size_t workspace_bytes(const race_args_t* a, bool backward) {
   return simt_plan(a, backward).bytes;
 }
 
+// ----------------------------------------------------------------------------- tensor
+template <int P>
+race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
+                        const CUtensorMap& tk, const CUtensorMap& tv, const float* W,
+                        const float* init, float* seg, float* num, cudaStream_t s) {
+  dim3 grid(prm.G, prm.n_rg, prm.H);
+  const size_t smem = tc::Smem::alloc;
+#define RACE_TC(MODE, NAME)                                                        \
+  do {                                                                             \
+    RACE_CU(set_smem(tc::k_sketch<P, MODE>, smem));                                \
+    RACE_LAUNCH(NAME, s);                                                          \
+    tc::k_sketch<P, MODE><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, W, init, seg, \
+                                                            num, prm);             \
+  } while (0)
+  if (mode == tc::kSweep) RACE_TC(tc::kSweep, "tc_causal_sweep");
+  else if (mode == tc::kBuild) RACE_TC(tc::kBuild, "tc_sketch_build");
+  else RACE_TC(tc::kReadout, "tc_readout");
+#undef RACE_TC
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+race_status_t tc_dispatch(int P, int mode, const tc::Params& prm, const CUtensorMap& tq,
+                          const CUtensorMap& tk, const CUtensorMap& tv, const float* W,
+                          const float* init, float* seg, float* num, cudaStream_t s) {
+  switch (P) {
+    case 6: return tc_launch<6>(mode, prm, tq, tk, tv, W, init, seg, num, s);
+    case 7: return tc_launch<7>(mode, prm, tq, tk, tv, W, init, seg, num, s);
+    case 8: return tc_launch<8>(mode, prm, tq, tk, tv, W, init, seg, num, s);
+  }
+  return RACE_ERR_UNSUPPORTED;
+}
+
+template <typename TO>
+race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, const void* v,
+                         const float* W, TO* out, char* ws, cudaStream_t s) {
+  tc::Plan pl = tc::make_plan(a);
+  CUtensorMap tq, tk, tv;
+  if (!tc::encode_tmap(&tq, q, a->N, a->H) || !tc::encode_tmap(&tk, k, a->N, a->H) ||
+      !tc::encode_tmap(&tv, v, a->N, a->H))
+    return RACE_ERR_CUDA;
+  float* num = reinterpret_cast<float*>(ws + pl.off_num);
+  float* seg = reinterpret_cast<float*>(ws + pl.off_seg);
+  float* init = reinterpret_cast<float*>(ws + pl.off_init);
+  const int64_t rows = (int64_t)a->H * a->N;
+  RACE_CU(cudaMemsetAsync(num, 0, (size_t)rows * kNumStride * sizeof(float), s));
+  tc::Params prm = pl.prm;
+  race_status_t st;
+  if (!a->causal || prm.G > 1) {
+    st = tc_dispatch(pl.P, tc::kBuild, prm, tq, tk, tv, W, init, seg, num, s);
+    if (st != RACE_OK) return st;
+    const int RD = prm.rows * tc::kNV;
+    {
+      RACE_LAUNCH("tc_chunk_scan", s);
+      simt::k_scan<<<dim3((RD + 255) / 256, prm.H * prm.n_rg), 256, 0, s>>>(
+          seg, init, RD, prm.G, a->causal ? 0 : 2);
+    }
+    RACE_CU(cudaGetLastError());
+    prm.have_init = 1;
+  }
+  st = tc_dispatch(pl.P, a->causal ? tc::kSweep : tc::kReadout, prm, tq, tk, tv, W, init,
+                   seg, num, s);
+  if (st != RACE_OK) return st;
+  {
+    RACE_LAUNCH("tc_normalize", s);
+    simt::k_normalize<TO><<<(unsigned)((rows + 3) / 4), 256, 0, s>>>(num, out, a->den, rows,
+                                                                      1.f / a->L);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
 // Scratch: the caller's, or stream-ordered memory of our own.
 struct Scratch {
   char* ptr = nullptr;
@@ -388,7 +461,11 @@ race_status_t forward_impl(const void* q, const void* k, const void* v, const fl
   Scratch sc;
   st = sc.acquire(a, workspace_bytes(a, false), s);
   if (st != RACE_OK) return st;
-  if (tensor) return tc::forward(a, q, k, v, W, out, sc.ptr, s);
+  if (tensor) {
+    if (a->out_dtype == RACE_BF16)
+      return tc_forward(a, q, k, v, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s);
+    return tc_forward(a, q, k, v, W, static_cast<float*>(out), sc.ptr, s);
+  }
   if (a->dtype == RACE_BF16) {
     auto* qq = static_cast<const __nv_bfloat16*>(q);
     auto* kk = static_cast<const __nv_bfloat16*>(k);

@@ -149,9 +149,17 @@ def test_backward_simt_parity(causal, N, dtype):
     dq, dk, dv, dW = ra.backward(g["q"], g["k"], g["v"], g["W"], wl.tau, causal, out,
                                  g["dout"], impl="simt")
     refs = _oracle_bwd(wl, x)
-    tol = 1e-4 if dtype == "fp32" else 1e-2
-    for name, got, ref in zip(("dq", "dk", "dv", "dW"), (dq, dk, dv, dW), refs):
-        err = np.abs(_np(got) - ref).max() / max(np.abs(ref).max(), 1e-30)
+    tol = 1e-4 if dtype == "fp32" else 4e-3
+    _check_grads((dq, dk, dv, dW), refs, tol)
+
+
+def _check_grads(got, refs, tol):
+    """max|dG| <= tol * max|G_ref| per gradient; a gradient that is exactly zero in
+    exact arithmetic (dq, dk at N = 1) is measured against the scale of dv."""
+    gscale = np.abs(refs[2]).max()
+    for name, g, ref in zip(("dq", "dk", "dv", "dW"), got, refs):
+        denom = max(np.abs(ref).max(), 1e-3 * gscale)
+        err = np.abs(_np(g) - ref).max() / denom
         assert err <= tol, (name, err)
 
 
