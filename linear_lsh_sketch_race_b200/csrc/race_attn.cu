@@ -13,6 +13,7 @@
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
 #include "tc_ptx.cuh"
+#include "tc_sweep.cuh"
 
 namespace race {
 
@@ -361,7 +362,13 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
     tc::k_sketch<P, MODE><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, W, init, seg, \
                                                             num, prm);             \
   } while (0)
-  if (mode == tc::kSweep) RACE_TC(tc::kSweep, "tc_causal_sweep");
+  if (mode == tc::kSweep && prm.rows == 256) {
+    constexpr int TABLES = 256 >> P;
+    RACE_CU(set_smem(tc::k_sweep<P, TABLES>, tc::SwSmem::alloc));
+    RACE_LAUNCH("tc_causal_sweep", s);
+    tc::k_sweep<P, TABLES><<<grid, tc::kSwThreads, tc::SwSmem::alloc, s>>>(tq, tk, tv, W, init,
+                                                                          num, prm);
+  } else if (mode == tc::kSweep) RACE_TC(tc::kSweep, "tc_causal_sweep_rows128");
   else if (mode == tc::kBuild) RACE_TC(tc::kBuild, "tc_sketch_build");
   else RACE_TC(tc::kReadout, "tc_readout");
 #undef RACE_TC
@@ -648,5 +655,15 @@ race_status_t race_timing_report(int i, const char** name, double* total_ms,
 }
 
 int64_t race_launch_count(void) { return launches::g_count.load(); }
+
+#ifdef RACE_SWEEP_TRACE
+// Copies the sweep timeline (see tc_sweep.cuh) to host memory `dst`; returns the
+// number of 64-bit stamps.
+int race_sweep_trace_read(unsigned long long* dst) {
+  cudaDeviceSynchronize();
+  cudaMemcpyFromSymbol(dst, tc::g_sweep_trace, sizeof(tc::g_sweep_trace));
+  return tc::kTraceChunks * tc::kTraceEvents;
+}
+#endif
 
 }  // extern "C"
