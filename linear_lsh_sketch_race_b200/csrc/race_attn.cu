@@ -14,6 +14,7 @@
 #include "tc_kernels.cuh"
 #include "tc_ptx.cuh"
 #include "tc_sweep.cuh"
+#include "tc_sweep256.cuh"
 
 namespace race {
 
@@ -352,7 +353,8 @@ size_t workspace_bytes(const race_args_t* a, bool backward) {
 template <int P>
 race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
                         const CUtensorMap& tk, const CUtensorMap& tv, const float* W,
-                        const float* init, float* seg, float* num, cudaStream_t s) {
+                        const float* init, float* seg, float* num, const float* inv_norms,
+                        int64_t inv_stride, cudaStream_t s) {
   dim3 grid(prm.G, prm.n_rg, prm.H);
   const size_t smem = tc::Smem::alloc;
 #define RACE_TC(MODE, NAME)                                                        \
@@ -362,7 +364,14 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
     tc::k_sketch<P, MODE><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, W, init, seg, \
                                                             num, prm);             \
   } while (0)
-  if (mode == tc::kSweep && prm.rows == 256) {
+  if (mode == tc::kSweep && P == 8 && prm.rows == 256 && inv_norms) {
+    CUtensorMap tnum;
+    if (!tc::encode_num_tmap(&tnum, num, prm.N, prm.H)) return RACE_ERR_CUDA;
+    RACE_CU(set_smem(tc::k_sweep256, tc::S8Smem::alloc));
+    RACE_LAUNCH("tc_causal_sweep", s);
+    tc::k_sweep256<<<grid, tc::kS8Threads, tc::S8Smem::alloc, s>>>(
+        tq, tk, tv, W, init, inv_norms, inv_stride, tnum, prm);
+  } else if (mode == tc::kSweep && prm.rows == 256) {
     constexpr int TABLES = 256 >> P;
     RACE_CU(set_smem(tc::k_sweep<P, TABLES>, tc::SwSmem::alloc));
     RACE_LAUNCH("tc_causal_sweep", s);
@@ -378,11 +387,12 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
 
 race_status_t tc_dispatch(int P, int mode, const tc::Params& prm, const CUtensorMap& tq,
                           const CUtensorMap& tk, const CUtensorMap& tv, const float* W,
-                          const float* init, float* seg, float* num, cudaStream_t s) {
+                          const float* init, float* seg, float* num, cudaStream_t s,
+                          const float* inv_norms = nullptr, int64_t inv_stride = 0) {
   switch (P) {
-    case 6: return tc_launch<6>(mode, prm, tq, tk, tv, W, init, seg, num, s);
-    case 7: return tc_launch<7>(mode, prm, tq, tk, tv, W, init, seg, num, s);
-    case 8: return tc_launch<8>(mode, prm, tq, tk, tv, W, init, seg, num, s);
+    case 6: return tc_launch<6>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, s);
+    case 7: return tc_launch<7>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, s);
+    case 8: return tc_launch<8>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, s);
   }
   return RACE_ERR_UNSUPPORTED;
 }
@@ -414,8 +424,17 @@ race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, con
     RACE_CU(cudaGetLastError());
     prm.have_init = 1;
   }
+  float* inv_norms = nullptr;
+  if (a->causal && pl.P == 8 && prm.rows == 256) {
+    inv_norms = reinterpret_cast<float*>(ws + pl.off_inv);
+    RACE_LAUNCH("tc_inv_norms", s);
+    tc::k_inv_norms<<<dim3((unsigned)((a->N + 255) / 256), 2 * a->H), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), inv_norms,
+        a->N, a->H, pl.inv_stride);
+  }
+  RACE_CU(cudaGetLastError());
   st = tc_dispatch(pl.P, a->causal ? tc::kSweep : tc::kReadout, prm, tq, tk, tv, W, init,
-                   seg, num, s);
+                   seg, num, s, inv_norms, pl.inv_stride);
   if (st != RACE_OK) return st;
   {
     RACE_LAUNCH("tc_normalize", s);

@@ -74,6 +74,28 @@ struct Tm {
                             intra = 416;  // intra: bf16 A operand, 64 columns
 };
 
+// One step of the Kronecker tree over planes: entries [0, HALF) become the products
+// with the "bit clear" factor and [HALF, 2*HALF) with the "bit set" factor.  A template
+// so every index is a compile-time constant (the array stays in registers).
+template <int HALF>
+__device__ __forceinline__ void kron_step(float* v, float set, float clear) {
+#pragma unroll
+  for (int c = 0; c < HALF; ++c) {
+    v[c + HALF] = v[c] * set;
+    v[c] = v[c] * clear;
+  }
+}
+
+// v[c] for c < 2^(P-FIRST): product over planes FIRST..P-1 of set (bit p-FIRST of c set)
+// or clear factors, times v[0] on entry.
+template <int FIRST, int P>
+__device__ __forceinline__ void kron_tree(float* v, const float* set, const float* clear) {
+  if constexpr (FIRST < P) {
+    kron_tree<FIRST, P - 1>(v, set, clear);
+    kron_step<(1 << (P - 1 - FIRST))>(v, set[P - 1], clear[P - 1]);
+  }
+}
+
 // --------------------------------------------------------------------------- helpers
 __device__ __forceinline__ void logistic_fast(float z, float& sp, float& sm) {
   const float e = __expf(-fabsf(z));
@@ -103,15 +125,7 @@ __device__ __forceinline__ void write_phi_rows(uint32_t tile, int t, int rows, i
       lo[b] = ((b & 1) ? sp[0] : sm[0]) * ((b & 2) ? sp[1] : sm[1]) * ((b & 4) ? sp[2] : sm[2]);
     float hi[NHI];
     hi[0] = valid ? 1.f : 0.f;
-#pragma unroll
-    for (int p = 3; p < P; ++p) {
-      const int half = 1 << (p - 3);
-#pragma unroll
-      for (int c = 0; c < half; ++c) {
-        hi[c + half] = hi[c] * sp[p];
-        hi[c] = hi[c] * sm[p];
-      }
-    }
+    kron_tree<3, P>(hi, sp, sm);
 #pragma unroll
     for (int c = 0; c < NHI; ++c) {
       const uint32_t addr = base + (uint32_t)((j * R) / 8 + c) * 128;
@@ -454,7 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 struct Plan {
   Params prm;
   int P;
-  size_t off_num, off_seg, off_init, bytes;
+  size_t off_num, off_seg, off_init, off_inv, bytes;
+  int64_t inv_stride;
 };
 
 inline bool supported(const race_args_t* a) {
@@ -498,6 +513,8 @@ inline Plan make_plan(const race_args_t* a) {
   pl.off_num = o;  o = al(o + (size_t)a->H * a->N * kNumStride * sizeof(float));
   pl.off_seg = o;  o = al(o + st);
   pl.off_init = o; o = al(o + st);
+  pl.inv_stride = ((a->N + kC - 1) / kC) * kC;  // per-head row stride: whole chunks
+  pl.off_inv = o;  o = al(o + 2 * (size_t)a->H * pl.inv_stride * sizeof(float));
   pl.bytes = o;
   return pl;
 }
@@ -522,6 +539,29 @@ inline bool encode_tmap(CUtensorMap* m, const void* base, int64_t N, int H) {
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D view [H][N][68] of the float32 output accumulators for TMA reductions: boxes of
+// 64 rows x 68 columns, rows beyond N of a head are dropped.
+inline bool encode_num_tmap(CUtensorMap* m, void* base, int64_t N, int H) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)kNumStride, (cuuint64_t)N, (cuuint64_t)H};
+  cuuint64_t strides[2] = {(cuuint64_t)kNumStride * 4, (cuuint64_t)N * kNumStride * 4};
+  cuuint32_t box[3] = {(cuuint32_t)kNumStride, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 

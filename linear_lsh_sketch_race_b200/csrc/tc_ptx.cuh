@@ -166,7 +166,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
 }
 
 // ------------------------------------------------------------------------ descriptors
-enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2 };
+enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle32B = 6 };
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and stride byte
 // offsets (all in 16-byte units), version 1, swizzle mode.

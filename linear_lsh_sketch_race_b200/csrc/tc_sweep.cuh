@@ -101,15 +101,7 @@ __device__ __forceinline__ void expand_half(uint32_t tile, int t, const float* s
       lo[b] = ((b & 1) ? sp[0] : sm[0]) * ((b & 2) ? sp[1] : sm[1]) * ((b & 4) ? sp[2] : sm[2]);
     float hi[16];
     hi[0] = valid * (HALF ? sp[P - 1] : sm[P - 1]);
-#pragma unroll
-    for (int p = 3; p < P - 1; ++p) {
-      const int half = 1 << (p - 3);
-#pragma unroll
-      for (int c = 0; c < half; ++c) {
-        hi[c + half] = hi[c] * sp[p];
-        hi[c] = hi[c] * sm[p];
-      }
-    }
+    kron_tree<3, P - 1>(hi, sp, sm);
 #pragma unroll
     for (int c = 0; c < 16; ++c) store_chunk(base + c * 128, hi[c], lo);
   } else {
@@ -125,15 +117,7 @@ __device__ __forceinline__ void expand_half(uint32_t tile, int t, const float* s
         lo[b] = ((b & 1) ? a[0] : b_[0]) * ((b & 2) ? a[1] : b_[1]) * ((b & 4) ? a[2] : b_[2]);
       float hi[R / 8];
       hi[0] = valid;
-#pragma unroll
-      for (int p = 3; p < P; ++p) {
-        const int half = 1 << (p - 3);
-#pragma unroll
-        for (int c = 0; c < half; ++c) {
-          hi[c + half] = hi[c] * a[p];
-          hi[c] = hi[c] * b_[p];
-        }
-      }
+      kron_tree<3, P>(hi, a, b_);
 #pragma unroll
       for (int c = 0; c < R / 8; ++c) store_chunk(base + (jj * (R / 8) + c) * 128, hi[c], lo);
     }
