@@ -168,15 +168,14 @@ __device__ __forceinline__ void store_state_row_bf16(uint32_t sbf, int row, cons
                  pack_bf16(v[nc * 8 + 6], v[nc * 8 + 7]));
 }
 
+// 80 consecutive columns of this thread's lane: five loads in flight, one wait.
 __device__ __forceinline__ void tmem_ld80(uint32_t taddr, float* v) {
-  uint32_t r[16];
+  uint32_t r[80];
 #pragma unroll
-  for (int b = 0; b < 5; ++b) {
-    tmem_ld16(taddr + b * 16, r);
-    tmem_ld_wait();
+  for (int b = 0; b < 5; ++b) tmem_ld16(taddr + b * 16, r + b * 16);
+  tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 16; ++e) v[b * 16 + e] = __uint_as_float(r[e]);
-  }
+  for (int e = 0; e < 80; ++e) v[e] = __uint_as_float(r[e]);
 }
 
 // --------------------------------------------------------------------------- kernel

@@ -52,10 +52,12 @@ static_assert(S8Smem::alloc <= 232448, "shared memory budget of one CTA");
 
 // Tensor memory.  qk holds the in-chunk QK (fp32, 128 columns); after masking, keys
 // 0-63 become bf16 A-operand columns qk+0..31 and keys 64-127 columns qk+64..95.  The
-// k projection of the next chunk lands in qk+112..127 once both groups have read QK.
+// projections of the next chunk land in the last 32 columns of the p(q) region (rows
+// 192-255 of p(q)) as soon as the QK of this chunk has read p(q); the q side writes
+// those rows of the next p(q) only after both sides have read the projections.
 struct S8Tm {
-  static constexpr uint32_t S0 = 0, S1 = 80, num = 160, phq = 240, pq = 368, qk = 384,
-                            intraA = 384, intraB = 448, pk = 496;
+  static constexpr uint32_t S0 = 0, S1 = 80, num = 160, phq = 240, pq = 336, pk = 352,
+                            qk = 368, intraA = 368, intraB = 432;
 };
 
 // 1/max(|x|, eps) of every row of q and k into out[side][h][stride] (side 0: q, 1: k);
@@ -329,6 +331,13 @@ __global__ void __launch_bounds__(kS8Threads, 1)
           umma_ts(tmem + S8Tm::qk, tmem + S8Tm::phq + s * 8,
                   d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, 1);
         umma_commit(bar + k8_QKDONE);      // QK complete; p(q) of this chunk no longer read
+        // next chunk's projections go into the p(q) columns just released (in issue
+        // order after the last MMA that reads p(q) of this chunk)
+        if (c + 1 < nchunks) {
+          if (!wait(k8_QKFULL0 + (st ^ 1), ((c + 1) >> 1) & 1)) break;
+          tc_fence_after();
+          issue_proj(c + 1);
+        }
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           umma_ss(tmem + S8Tm::S1, d_up1 + 128 * s, d_vone + vstep * s, id_up, 1);
@@ -337,12 +346,6 @@ __global__ void __launch_bounds__(kS8Threads, 1)
         if (!wait(k8_CONV, par)) break;
         SW_TRACE(c, 5);
         tc_fence_after();
-        // next chunk's projections (pk shares columns with the converted QK)
-        if (c + 1 < nchunks) {
-          if (!wait(k8_QKFULL0 + (st ^ 1), ((c + 1) >> 1) & 1)) break;
-          tc_fence_after();
-          issue_proj(c + 1);
-        }
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           umma_ts(tmem + S8Tm::num,
@@ -449,6 +452,7 @@ __global__ void __launch_bounds__(kS8Threads, 1)
         tc_fence_after();
 #pragma unroll
         for (int blk = 0; blk < 8; ++blk) {
+          if (blk == 6 && !wait(k8_PROJFREE, par)) break;   // rows 192-255 hold projections
           uint32_t v16[16];
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
@@ -492,18 +496,16 @@ __global__ void __launch_bounds__(kS8Threads, 1)
       tc_fence_after();
       const uint32_t src = tmem + lane_off + S8Tm::qk + grp * 64;
       const uint32_t dst = tmem + lane_off + (grp ? S8Tm::intraB : S8Tm::intraA);
-      uint32_t out32[32];
+      uint32_t out32[32], qk64[64];
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        tmem_ld16(src + cb * 16, r);
-        tmem_ld_wait();
+      for (int cb = 0; cb < 4; ++cb) tmem_ld16(src + cb * 16, qk64 + cb * 16);
+      tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j0 = grp * 64 + cb * 16 + 2 * e;
-          const float a0 = (j0 <= t) ? __uint_as_float(r[2 * e]) : 0.f;
-          const float a1 = (j0 + 1 <= t) ? __uint_as_float(r[2 * e + 1]) : 0.f;
-          out32[cb * 8 + e] = pack_bf16(a0, a1);
-        }
+      for (int e = 0; e < 32; ++e) {
+        const int j0 = grp * 64 + 2 * e;
+        const float a0 = (j0 <= t) ? __uint_as_float(qk64[2 * e]) : 0.f;
+        const float a1 = (j0 + 1 <= t) ? __uint_as_float(qk64[2 * e + 1]) : 0.f;
+        out32[e] = pack_bf16(a0, a1);
       }
       tmem_st16(dst, out32);
       tmem_st16(dst + 16, out32 + 16);
