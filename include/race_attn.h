@@ -59,8 +59,10 @@ typedef enum {
   RACE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d != 64)             */
   RACE_ERR_WORKSPACE = 3,     /* caller workspace too small or allocation failed     */
   RACE_ERR_CUDA = 4,          /* a CUDA runtime call or a launch failed              */
-  RACE_ERR_DEVICE_STATUS = 5  /* a kernel raised its device status flag (a bounded   */
+  RACE_ERR_DEVICE_STATUS = 5, /* a kernel raised its device status flag (a bounded  */
                               /* wait gave up, or an index check failed)             */
+  RACE_ERR_SCRATCH_LIMIT = 6  /* race_forward_noalloc: the problem needs more scratch */
+                              /* than RACE_NOALLOC_SCRATCH_BYTES                     */
 } race_status_t;
 
 typedef enum { RACE_BF16 = 0, RACE_FP32 = 1 } race_dtype_t;
@@ -130,6 +132,37 @@ race_status_t race_backward_ex(const void *q, const void *k, const void *v,
                                const float *W, const void *out, const void *dout,
                                void *dq, void *dk, void *dv, float *dW,
                                const race_args_t *a, race_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * race_forward_noalloc — the forward of race_forward_ex computed without allocating
+ * any memory.  The paper has no counterpart: this is a deployment aid for callers that
+ * cannot allocate device memory at call time, e.g. a serving process that reserves
+ * all free HBM for its caches at start-up (any later cudaMalloc fails or fragments the
+ * reservation) or a latency-bound loop that must not enter the allocator, which can
+ * synchronise or grow its pool.
+ *
+ * Arguments, layouts and results are those of race_forward_ex; a->workspace and
+ * a->workspace_bytes are ignored.  The scratch is instead one fixed device array of
+ * RACE_NOALLOC_SCRATCH_BYTES that is part of the library's loaded module (one per
+ * device).  No cudaMalloc, cudaMallocAsync or other allocating routine is called; the
+ * call clears the parts of the array that must start at zero on `stream` itself.
+ *
+ * Set-up: the first call on each device looks up the array's device address (with
+ * that device current) and may load the module there.  Make that first call before
+ * any stream capture begins.
+ *
+ * Concurrency: all calls on one device share the array.  Calls that can overlap in
+ * time (different streams, or different host threads without ordering) race on it and
+ * give wrong results; order them on one stream.
+ *
+ * Errors: RACE_ERR_SCRATCH_LIMIT, before any device work, when
+ * race_workspace_size(a, 0) exceeds RACE_NOALLOC_SCRATCH_BYTES; RACE_ERR_CUDA when the
+ * address look-up fails; otherwise the statuses of race_forward_ex.
+ * ------------------------------------------------------------------------------ */
+#define RACE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+race_status_t race_forward_noalloc(const void *q, const void *k, const void *v,
+                                   const float *W, void *out, const race_args_t *a,
+                                   race_stream_t stream);
 
 /* Scratch bytes the *_ex calls need for `a` (backward != 0: the backward).  Writes 0
  * and returns an error status for invalid or unsupported arguments.  Host only; no

@@ -535,6 +535,42 @@ race_status_t backward_impl(const void* q, const void* k, const void* v, const f
 #undef RACE_BWD
 }
 
+// ------------------------------------------------------------ allocation-free forward
+// Scratch of race_forward_noalloc.  Some callers cannot allocate device memory at call
+// time: a serving process that reserved all free HBM for its caches at start-up, or a
+// latency-bound loop that must not enter an allocator (which can synchronise or grow
+// its pool).  For them the scratch is this fixed array, part of the loaded module: it
+// costs RACE_NOALLOC_SCRATCH_BYTES on every device the module is loaded on and is
+// shared by all calls on that device, so overlapping calls race.
+static __device__ __align__(256) char g_noalloc_scratch[RACE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+char* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device
+// (the look-up may load the module there, so it belongs before any stream capture).
+race_status_t noalloc_scratch(char** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return RACE_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return RACE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();
+      return RACE_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<char*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return RACE_OK;
+}
+
 }  // namespace
 }  // namespace race
 
@@ -587,6 +623,24 @@ race_status_t race_backward_ex(const void* q, const void* k, const void* v,
                                race_stream_t stream) {
   return backward_impl(q, k, v, W, out, dout, dq, dk, dv, dW, a,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+race_status_t race_forward_noalloc(const void* q, const void* k, const void* v,
+                                   const float* W, void* out, const race_args_t* a,
+                                   race_stream_t stream) {
+  if (!a) return RACE_ERR_INVALID_ARG;
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  if (workspace_bytes(a, false) > RACE_NOALLOC_SCRATCH_BYTES) return RACE_ERR_SCRATCH_LIMIT;
+  char* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != RACE_OK) return st;
+  // The forward clears its accumulators itself (every path memsets or fully writes
+  // the scratch it reads), so the array needs no clearing between calls.
+  race_args_t b = *a;
+  b.workspace = ws;
+  b.workspace_bytes = RACE_NOALLOC_SCRATCH_BYTES;
+  return forward_impl(q, k, v, W, out, &b, reinterpret_cast<cudaStream_t>(stream));
 }
 
 race_status_t race_workspace_size(const race_args_t* a, int backward, size_t* bytes) {
@@ -647,6 +701,9 @@ const char* race_status_string(race_status_t s) {
     case RACE_ERR_WORKSPACE: return "RACE_ERR_WORKSPACE: scratch too small or allocation failed";
     case RACE_ERR_CUDA: return "RACE_ERR_CUDA: CUDA call or launch failed";
     case RACE_ERR_DEVICE_STATUS: return "RACE_ERR_DEVICE_STATUS: a kernel raised the device status flag";
+    case RACE_ERR_SCRATCH_LIMIT:
+      return "RACE_ERR_SCRATCH_LIMIT: problem needs more scratch than the fixed "
+             "RACE_NOALLOC_SCRATCH_BYTES array of race_forward_noalloc";
   }
   return "unknown race_status_t";
 }

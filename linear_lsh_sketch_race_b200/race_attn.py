@@ -6,7 +6,8 @@ computation runs in the library's kernels.  A missing or unloadable library rais
 immediately; there is no fallback.
 
 The C entry points keep their names: ``race_forward``, ``race_backward``,
-``race_forward_ex``, ``race_backward_ex``, ``race_workspace_size``, ``race_hash``,
+``race_forward_ex``, ``race_backward_ex``, ``race_forward_noalloc``,
+``race_workspace_size``, ``race_hash``,
 ``race_device_status``, ``race_status_string``, ``race_version``, ``race_args_init``.
 ``forward``/``backward``/``hash`` are conveniences that allocate outputs.
 """
@@ -22,7 +23,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librace_attn.so")
 
 RACE_OK, RACE_ERR_INVALID_ARG, RACE_ERR_UNSUPPORTED, RACE_ERR_WORKSPACE, \
-    RACE_ERR_CUDA, RACE_ERR_DEVICE_STATUS = range(6)
+    RACE_ERR_CUDA, RACE_ERR_DEVICE_STATUS, RACE_ERR_SCRATCH_LIMIT = range(7)
+RACE_NOALLOC_SCRATCH_BYTES = 64 << 20
 RACE_BF16, RACE_FP32 = 0, 1
 RACE_IMPL_AUTO, RACE_IMPL_SIMT, RACE_IMPL_TENSOR = 0, 1, 2
 _IMPLS = {"auto": RACE_IMPL_AUTO, "simt": RACE_IMPL_SIMT, "tensor": RACE_IMPL_TENSOR}
@@ -30,7 +32,7 @@ _IMPLS = {"auto": RACE_IMPL_AUTO, "simt": RACE_IMPL_SIMT, "tensor": RACE_IMPL_TE
 EXPORTED = ("race_args_init", "race_forward", "race_backward", "race_forward_ex",
             "race_backward_ex", "race_workspace_size", "race_hash", "race_device_status",
             "race_status_string", "race_version", "race_timing_enable",
-            "race_timing_report", "race_launch_count")
+            "race_timing_report", "race_launch_count", "race_forward_noalloc")
 
 
 class RaceArgs(ctypes.Structure):
@@ -78,6 +80,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_backward.argtypes = [vp] * 10 + [i64, i32, i32, i32, i32, f32, i32, vp]
     lib.race_forward_ex.argtypes = [vp, vp, vp, vp, vp, pargs, vp]
     lib.race_backward_ex.argtypes = [vp] * 10 + [pargs, vp]
+    lib.race_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, pargs, vp]
     lib.race_workspace_size.argtypes = [pargs, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.race_hash.argtypes = [vp, vp, vp, pargs, vp]
     lib.race_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -91,7 +94,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_launch_count.argtypes = []
     lib.race_launch_count.restype = i64
     for name in ("race_forward", "race_backward", "race_forward_ex", "race_backward_ex",
-                 "race_workspace_size", "race_hash", "race_device_status",
+                 "race_forward_noalloc", "race_workspace_size", "race_hash", "race_device_status",
                  "race_timing_enable", "race_timing_report"):
         getattr(lib, name).restype = i32
     lib.race_version.restype = i32
@@ -154,6 +157,12 @@ def race_backward(q, k, v, W, out, dout, dq, dk, dv, dW, N, H, d, L, P, tau, cau
 def race_forward_ex(q, k, v, W, out, args: RaceArgs, stream=None):
     _check(load().race_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out),
                                   ctypes.byref(args), _stream(stream)), "race_forward_ex")
+
+
+def race_forward_noalloc(q, k, v, W, out, args: RaceArgs, stream=None):
+    _check(load().race_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out),
+                                       ctypes.byref(args), _stream(stream)),
+           "race_forward_noalloc")
 
 
 def race_backward_ex(q, k, v, W, out, dout, dq, dk, dv, dW, args: RaceArgs, stream=None):
