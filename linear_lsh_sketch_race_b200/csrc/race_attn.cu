@@ -15,6 +15,7 @@
 #include "tc_ptx.cuh"
 #include "tc_sweep.cuh"
 #include "tc_sweep256.cuh"
+#include "tc_backward.cuh"
 
 namespace race {
 
@@ -344,8 +345,19 @@ bool use_tensor_path(const race_args_t* a) {
   return tc::supported(a);
 }
 
+bool tc_backward_supported(const race_args_t* a);
+struct BwPlan;
+size_t bw_plan_bytes(const race_args_t* a);
+
+bool use_tensor_backward(const race_args_t* a) {
+  if (a->impl == RACE_IMPL_SIMT) return false;
+  if (a->dtype != RACE_BF16) return false;
+  return tc_backward_supported(a);
+}
+
 size_t workspace_bytes(const race_args_t* a, bool backward) {
   if (!backward && use_tensor_path(a)) return tc::forward_workspace(a);
+  if (backward && use_tensor_backward(a)) return bw_plan_bytes(a);
   return simt_plan(a, backward).bytes;
 }
 
@@ -397,9 +409,10 @@ race_status_t tc_dispatch(int P, int mode, const tc::Params& prm, const CUtensor
   return RACE_ERR_UNSUPPORTED;
 }
 
-template <typename TO>
-race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, const void* v,
-                         const float* W, TO* out, char* ws, cudaStream_t s) {
+// Forward accumulators num[h][n][0..64] (unnormalised, den' in column 64) in the
+// forward plan's scratch.
+race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k, const void* v,
+                             const float* W, char* ws, float** num_out, cudaStream_t s) {
   tc::Plan pl = tc::make_plan(a);
   CUtensorMap tq, tk, tv;
   if (!tc::encode_tmap(&tq, q, a->N, a->H) || !tc::encode_tmap(&tk, k, a->N, a->H) ||
@@ -436,10 +449,237 @@ race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, con
   st = tc_dispatch(pl.P, a->causal ? tc::kSweep : tc::kReadout, prm, tq, tk, tv, W, init,
                    seg, num, s, inv_norms, pl.inv_stride);
   if (st != RACE_OK) return st;
+  *num_out = num;
+  return RACE_OK;
+}
+
+template <typename TO>
+race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, const void* v,
+                         const float* W, TO* out, char* ws, cudaStream_t s) {
+  float* num = nullptr;
+  race_status_t st = tc_forward_num(a, q, k, v, W, ws, &num, s);
+  if (st != RACE_OK) return st;
+  const int64_t rows = (int64_t)a->H * a->N;
   {
     RACE_LAUNCH("tc_normalize", s);
     simt::k_normalize<TO><<<(unsigned)((rows + 3) / 4), 256, 0, s>>>(num, out, a->den, rows,
                                                                       1.f / a->L);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+// ----------------------------------------------------------------------------- tensor backward
+// Row groups of 256 sketch rows (L*R a multiple of 256) and L*P <= 256.
+bool tc_backward_supported(const race_args_t* a) {
+  if (!tc::supported(a)) return false;
+  const int64_t LR = (int64_t)a->L << a->P;
+  return LR % 256 == 0 && (int64_t)a->L * a->P <= tc::kMaxLP;
+}
+
+struct BwPlan {
+  tc::Params prm;
+  int fin_blocks;
+  size_t off_fwd, off_gh, off_gdot, off_rq, off_rk, off_rg, off_duq, off_duk, off_seg,
+      off_init, off_part, bytes;
+};
+
+BwPlan make_bw_plan(const race_args_t* a) {
+  BwPlan b;
+  tc::Params& p = b.prm;
+  p.N = a->N;
+  p.H = a->H;
+  p.L = a->L;
+  p.R = 1 << a->P;
+  p.rows = 256;
+  p.tables = 256 / p.R;
+  p.np = ((p.tables * a->P + 15) / 16) * 16;
+  p.n_rg = (a->L * p.R) / 256;
+  const int64_t units = (int64_t)a->H * p.n_rg;
+  const int64_t tiles = (a->N + tc::kC - 1) / tc::kC;
+  int64_t G = a->causal ? std::max<int64_t>(1, kPlanSMs / units)
+                        : std::max<int64_t>(1, (kPlanSMs + units - 1) / units);
+  G = std::min<int64_t>(G, tiles);
+  p.seg_len = ((tiles + G - 1) / G) * tc::kC;
+  p.G = (int)((a->N + p.seg_len - 1) / p.seg_len);
+  p.two_over_tau = 2.0f / a->tau;
+  p.have_init = 0;
+  const int64_t rows = (int64_t)a->H * a->N;
+  const int LP = a->L * a->P;
+  b.fin_blocks = (int)std::max<int64_t>(1, std::min<int64_t>(4 * kPlanSMs, (rows + tc::kFinTok - 1) / tc::kFinTok));
+  const size_t st = (size_t)a->H * p.n_rg * p.G * 256 * tc::kNV * sizeof(float);
+  const size_t xb = (size_t)rows * kD * sizeof(__nv_bfloat16);
+  size_t o = 0;
+  b.off_fwd = o;  o = align_up(o + tc::forward_workspace(a));
+  b.off_gh = o;   o = align_up(o + xb);
+  b.off_gdot = o; o = align_up(o + (size_t)rows * sizeof(float));
+  b.off_rq = b.off_rk = b.off_rg = o;
+  if (a->causal) {
+    b.off_rq = o; o = align_up(o + xb);
+    b.off_rk = o; o = align_up(o + xb);
+    b.off_rg = o; o = align_up(o + xb);
+  }
+  b.off_duq = o;  o = align_up(o + (size_t)rows * LP * sizeof(float));
+  b.off_duk = o;  o = align_up(o + (size_t)rows * LP * sizeof(float));
+  b.off_seg = o;  o = align_up(o + st);
+  b.off_init = o; o = align_up(o + st);
+  b.off_part = o; o = align_up(o + 2 * (size_t)b.fin_blocks * LP * kD * sizeof(float));
+  b.bytes = o;
+  return b;
+}
+
+size_t bw_plan_bytes(const race_args_t* a) { return make_bw_plan(a).bytes; }
+
+template <int P>
+race_status_t bw_launch(int mode, bool rev, const tc::Params& prm, const CUtensorMap& xa,
+                        const CUtensorMap& xb, const CUtensorMap& fa, const CUtensorMap& fb,
+                        const float* ea, const float* eb, const float* W, const float* init,
+                        float* seg, float* du, const char* name, cudaStream_t s) {
+  dim3 grid(prm.G, prm.n_rg, prm.H);
+  const size_t smem = tc::BwSmem::alloc;
+#define RACE_BW(MODE, REV)                                                                 \
+  do {                                                                                     \
+    RACE_CU(set_smem(tc::k_bwd_phi<P, MODE, REV>, smem));                                  \
+    RACE_LAUNCH(name, s);                                                                  \
+    tc::k_bwd_phi<P, MODE, REV><<<grid, tc::kBwThreads, smem, s>>>(xa, xb, fa, fb, ea, eb, \
+                                                                   W, init, seg, du, prm); \
+  } while (0)
+  if (mode == tc::kBuild) RACE_BW(tc::kBuild, false);
+  else if (mode == tc::kReadout) RACE_BW(tc::kReadout, false);
+  else if (rev) RACE_BW(tc::kSweep, true);
+  else RACE_BW(tc::kSweep, false);
+#undef RACE_BW
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+race_status_t bw_dispatch(int P, int mode, bool rev, const tc::Params& prm,
+                          const CUtensorMap& xa, const CUtensorMap& xb, const CUtensorMap& fa,
+                          const CUtensorMap& fb, const float* ea, const float* eb,
+                          const float* W, const float* init, float* seg, float* du,
+                          const char* name, cudaStream_t s) {
+  switch (P) {
+    case 6: return bw_launch<6>(mode, rev, prm, xa, xb, fa, fb, ea, eb, W, init, seg, du, name, s);
+    case 7: return bw_launch<7>(mode, rev, prm, xa, xb, fa, fb, ea, eb, W, init, seg, du, name, s);
+    case 8: return bw_launch<8>(mode, rev, prm, xa, xb, fa, fb, ea, eb, W, init, seg, du, name, s);
+  }
+  return RACE_ERR_UNSUPPORTED;
+}
+
+template <typename TO>
+race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                          const __nv_bfloat16* v, const float* W, const TO* out,
+                          const __nv_bfloat16* dout, __nv_bfloat16* dq, __nv_bfloat16* dk,
+                          __nv_bfloat16* dv, float* dW, char* ws, cudaStream_t s) {
+  const BwPlan pl = make_bw_plan(a);
+  const int64_t rows = (int64_t)a->H * a->N;
+  const int LP = a->L * a->P;
+  char* fws = ws + pl.off_fwd;
+  auto* gh = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_gh);
+  float* gdot = reinterpret_cast<float*>(ws + pl.off_gdot);
+  float* duq = reinterpret_cast<float*>(ws + pl.off_duq);
+  float* duk = reinterpret_cast<float*>(ws + pl.off_duk);
+  float* seg = reinterpret_cast<float*>(ws + pl.off_seg);
+  float* init = reinterpret_cast<float*>(ws + pl.off_init);
+  float* partq = reinterpret_cast<float*>(ws + pl.off_part);
+  float* partk = partq + (size_t)pl.fin_blocks * LP * kD;
+  race_status_t st;
+  // ---- den' (recomputed by a forward when not saved) and g''
+  float* num = nullptr;
+  if (!a->den) {
+    st = tc_forward_num(a, q, k, v, W, fws, &num, s);
+    if (st != RACE_OK) return st;
+  }
+  {
+    RACE_LAUNCH("tc_bwd_prep", s);
+    tc::k_bwd_prep<__nv_bfloat16, TO><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+        dout, out, num, a->den, gh, gdot, rows, (float)a->L);
+  }
+  RACE_CU(cudaGetLastError());
+  CUtensorMap xq, xk, fv, fg;
+  if (!tc::encode_tmap(&xq, q, a->N, a->H) || !tc::encode_tmap(&xk, k, a->N, a->H) ||
+      !tc::encode_feat_tmap(&fv, v, a->N, a->H) || !tc::encode_feat_tmap(&fg, gh, a->N, a->H))
+    return RACE_ERR_CUDA;
+  const int mode = a->causal ? tc::kSweep : tc::kReadout;
+  const int RD = 256 * tc::kNV;
+  // ---- q side: dP(q) = g'' S^T + mask(g'' [v|1]^T) p(k), S over keys j <= i
+  tc::Params prm = pl.prm;
+  if (!a->causal || prm.G > 1) {
+    st = bw_dispatch(a->P, tc::kBuild, false, prm, xk, xk, fv, fv, nullptr, nullptr, W, init,
+                     seg, nullptr, "tc_bwd_build_k", s);
+    if (st != RACE_OK) return st;
+    {
+      RACE_LAUNCH("tc_chunk_scan", s);
+      simt::k_scan<<<dim3((RD + 255) / 256, prm.H * prm.n_rg), 256, 0, s>>>(
+          seg, init, RD, prm.G, a->causal ? 0 : 2);
+    }
+    RACE_CU(cudaGetLastError());
+    prm.have_init = 1;
+  }
+  st = bw_dispatch(a->P, mode, false, prm, xq, xk, fg, fv, gdot, nullptr, W, init, seg, duq,
+                   "tc_bwd_q", s);
+  if (st != RACE_OK) return st;
+  // ---- k side: dP(k) = [v|1] T^T + mask([v|1] g''^T) p(q), T over queries i >= j
+  prm = pl.prm;
+  if (!a->causal || prm.G > 1) {
+    st = bw_dispatch(a->P, tc::kBuild, false, prm, xq, xq, fg, fg, nullptr, gdot, W, init,
+                     seg, nullptr, "tc_bwd_build_q", s);
+    if (st != RACE_OK) return st;
+    {
+      RACE_LAUNCH("tc_chunk_scan", s);
+      simt::k_scan<<<dim3((RD + 255) / 256, prm.H * prm.n_rg), 256, 0, s>>>(
+          seg, init, RD, prm.G, a->causal ? 1 : 2);
+    }
+    RACE_CU(cudaGetLastError());
+    prm.have_init = 1;
+  }
+  st = bw_dispatch(a->P, mode, a->causal != 0, prm, xk, xq, fv, fg, nullptr, gdot, W, init,
+                   seg, duk, "tc_bwd_k", s);
+  if (st != RACE_OK) return st;
+  // ---- dv_j = sum_{i >= j} w_ij g_i/den'_i: the forward sweep with queries k, keys q and
+  //      values g'' (sequence reversed for the causal case)
+  race_args_t av = *a;
+  av.den = nullptr;
+  float* vnum = nullptr;
+  if (a->causal) {
+    auto* rq = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_rq);
+    auto* rk = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_rk);
+    auto* rg = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_rg);
+    const unsigned blocks = (unsigned)((rows * 8 + 255) / 256);
+    {
+      RACE_LAUNCH("tc_bwd_reverse", s);
+      tc::k_reverse_rows<<<blocks, 256, 0, s>>>(q, rq, a->N, a->H);
+      tc::k_reverse_rows<<<blocks, 256, 0, s>>>(k, rk, a->N, a->H);
+      tc::k_reverse_rows<<<blocks, 256, 0, s>>>(gh, rg, a->N, a->H);
+    }
+    RACE_CU(cudaGetLastError());
+    st = tc_forward_num(&av, rk, rq, rg, W, fws, &vnum, s);
+  } else {
+    st = tc_forward_num(&av, k, q, gh, W, fws, &vnum, s);
+  }
+  if (st != RACE_OK) return st;
+  {
+    RACE_LAUNCH("tc_bwd_dv_out", s);
+    tc::k_dv_out<__nv_bfloat16><<<(unsigned)((rows * kD + 255) / 256), 256, 0, s>>>(
+        vnum, dv, a->N, a->H, a->causal);
+  }
+  RACE_CU(cudaGetLastError());
+  // ---- dq, dk through the projections and the normalisation; dW
+  const size_t fsm = tc::finalize_smem(LP);
+  RACE_CU(set_smem(tc::k_bwd_finalize<__nv_bfloat16>, fsm));
+  {
+    RACE_LAUNCH("tc_bwd_finalize", s);
+    tc::k_bwd_finalize<__nv_bfloat16><<<pl.fin_blocks, 256, fsm, s>>>(q, duq, W, dq, partq,
+                                                                       rows, a->L, a->P);
+    tc::k_bwd_finalize<__nv_bfloat16><<<pl.fin_blocks, 256, fsm, s>>>(k, duk, W, dk, partk,
+                                                                       rows, a->L, a->P);
+  }
+  RACE_CU(cudaGetLastError());
+  const int nW = a->L * kD * a->P;
+  {
+    RACE_LAUNCH("tc_bwd_dW_reduce", s);
+    tc::k_bwd_dw_reduce<<<(nW + 255) / 256, 256, 0, s>>>(partq, partk, pl.fin_blocks, dW,
+                                                         a->L, a->P);
   }
   RACE_CU(cudaGetLastError());
   return RACE_OK;
@@ -517,10 +757,25 @@ race_status_t backward_impl(const void* q, const void* k, const void* v, const f
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return RACE_ERR_INVALID_ARG;
   if (a->den && !aligned16(a->den)) return RACE_ERR_INVALID_ARG;
-  if (a->impl == RACE_IMPL_TENSOR) return RACE_ERR_UNSUPPORTED;
+  const bool tensor = use_tensor_backward(a);
+  if (a->impl == RACE_IMPL_TENSOR && !tensor) return RACE_ERR_UNSUPPORTED;
   Scratch sc;
   st = sc.acquire(a, workspace_bytes(a, true), s);
   if (st != RACE_OK) return st;
+  if (tensor) {
+    auto* qq = static_cast<const __nv_bfloat16*>(q);
+    auto* kk = static_cast<const __nv_bfloat16*>(k);
+    auto* vv = static_cast<const __nv_bfloat16*>(v);
+    auto* gg = static_cast<const __nv_bfloat16*>(dout);
+    auto* dqq = static_cast<__nv_bfloat16*>(dq);
+    auto* dkk = static_cast<__nv_bfloat16*>(dk);
+    auto* dvv = static_cast<__nv_bfloat16*>(dv);
+    if (a->out_dtype == RACE_BF16)
+      return tc_backward(a, qq, kk, vv, W, static_cast<const __nv_bfloat16*>(out), gg, dqq,
+                         dkk, dvv, dW, sc.ptr, s);
+    return tc_backward(a, qq, kk, vv, W, static_cast<const float*>(out), gg, dqq, dkk, dvv,
+                       dW, sc.ptr, s);
+  }
 #define RACE_BWD(T, TO)                                                                  \
   return simt_backward<T, TO>(a, static_cast<const T*>(q), static_cast<const T*>(k),     \
                               static_cast<const T*>(v), W, static_cast<const TO*>(out),  \

@@ -1,0 +1,684 @@
+// Tensor-core (tcgen05) backward of RACE attention for row groups of 256 sketch rows
+// (one table at R = 256, 256/R tables below).
+//
+// Notation (kernel units: p = unscaled corner probabilities, den' = L * den):
+//   g''_i = [g_i / den'_i , -(g_i . o_i) / den'_i]       (80 wide: the last entry as a
+//                                                          bf16 hi + lo pair, then zeros)
+//   dw_ij = g''_i . [v_j ; 1]                             (gradient of the weight w_ij)
+//   dP(q_i) = sum_{j <= i} dw_ij p(k_j) = S_i g''_i        S_i = sum_{j <= i} p(k_j)[v_j;1]^T
+//   dP(k_j) = sum_{i >= j} dw_ij p(q_i) = T_j [v_j ; 1]    T_j = sum_{i >= j} p(q_i) g''_i^T
+// Both are the same computation with the roles of the two sides exchanged and the
+// sweep reversed: a side "a" whose corner gradients are wanted, with 80-wide features
+// X, and a side "b" with features Y whose p(b) builds the state:
+//   dP_a = X S^T + mask(X Y^T) p(b),   S += p(b)^T Y
+//   q pass: a = q, X = g'', b = k, Y = [v | 1]; forward order, keys j <= i
+//   k pass: a = k, X = [v | 1], b = q, Y = g''; reverse order, queries i >= j
+// The soft hash backward then gives, per table and plane ([JA] §2.1 soft
+// bucketization; the softmax over corners factorises into logistic pairs),
+//   du_p = (2/tau) (sum_{b: bit p of b set} p_b dP_b - s_p sum_b p_b dP_b),
+//   s_p = sigma(2 u_p / tau),
+// written per token to du[h][n][L*P]; the projection transposes and the
+// normalisation Jacobian run in k_bwd_finalize.
+//
+// One CTA sweeps one segment of one row group of one head: TMA loads the x tiles
+// (128B swizzle) and the feature tiles (32-byte swizzle, 4 boxes of 16 columns plus a
+// fifth atom holding the extra column); tcgen05 computes the projections, X Y^T, the
+// corner gradients (two halves of 128 rows) and the state update; the CUDA-core warps
+// expand p(b), mask and round X Y^T, run the hash backward and keep the bf16 copy of S.
+#pragma once
+
+#include "tc_kernels.cuh"
+
+namespace race {
+namespace tc {
+
+constexpr int kBwThreads = 160;  // warps 0-3: CUDA-core work (TMEM lane = token row); warp 4: issuer
+
+struct BwSmem {
+  static constexpr uint32_t xa = 0;        // 128 x 64 bf16, 128B swizzle (TMA)
+  static constexpr uint32_t xb = 16384;
+  static constexpr uint32_t fa = 32768;    // 5 atoms of 128 rows x 32 B, 32B swizzle
+  static constexpr uint32_t fb = 53248;
+  static constexpr uint32_t phb = 73728;   // p(b): 128 tokens x 256 rows, core-matrix layout
+  static constexpr uint32_t sbf = 139264;  // state as bf16 hi, 256 x 80, core-matrix layout
+  static constexpr uint32_t sbl = 180224;  // and the bf16 rest (S - hi)
+  static constexpr uint32_t whi = 221184;  // projection operand, up to 32 x 64 bf16
+  static constexpr uint32_t wlo = 225280;
+  static constexpr uint32_t bars = 229376;
+  static constexpr uint32_t total = bars + 16 * 8;
+  static constexpr uint32_t alloc = total + 1024;
+};
+static_assert(BwSmem::alloc <= 232448, "shared memory budget of one CTA");
+
+// Tensor-memory columns.  dw (float32, 128 keys) is rounded in place to the bf16 A
+// operand intra (64 columns).
+struct BwTm {
+  static constexpr uint32_t S0 = 0, S1 = 80, dp = 160, dw = 288, intra = 288, pa = 416,
+                            pb = 448;
+};
+
+enum BwBar : int {
+  kbTMA = 0, kbPROJ, kbPHI, kbDW, kbINTRA, kbDP, kbDPFREE, kbUP, kbFREE, kbCOUNT
+};
+
+// Extra feature columns of token row t in atom 4 of a 32B-swizzled feature tile.  The
+// 16 columns 64..79 are [e_hi, e_lo, 0, ...] with e = e_hi + e_lo split into two bf16
+// values on the g'' side, and [1, 1, 0, ...] on the [v | 1] side, so that their product
+// keeps -(g . o)/den' to about 16 bits: it nearly cancels g . v / den' in dw_ij.  Zero
+// for tokens past the end.  The two 16-byte halves of a 32-byte row are swapped on rows
+// 4-7 of each 8-row group.
+__device__ __forceinline__ void store_extra_cols(uint32_t tile, int t, const float* e,
+                                                 size_t idx, bool valid) {
+  float c0 = 0.f, c1 = 0.f;
+  if (valid) {
+    if (e) {
+      const float x = e[idx];
+      c0 = __bfloat162float(__float2bfloat16_rn(x));
+      c1 = x - c0;
+    } else {
+      c0 = c1 = 1.f;
+    }
+  }
+  const uint32_t row = tile + 4 * 4096 + t * 32;
+  const uint32_t first = ((t >> 2) & 1) << 4;
+  st_shared_v4(row + first, pack_bf16(c0, c1), 0u, 0u, 0u);
+  st_shared_v4(row + (first ^ 16), 0u, 0u, 0u, 0u);
+}
+
+// State row r as bf16 hi and bf16 lo = row - hi (X S^T adds both: the products with
+// g'' cancel to a small fraction of the state's size, so one bf16 rounding is too coarse).
+__device__ __forceinline__ void store_state_row_split(uint32_t hi_base, uint32_t lo_base, int r,
+                                                      const float* v) {
+  float lo[kNV];
+#pragma unroll
+  for (int c = 0; c < kNV; ++c) lo[c] = v[c] - __bfloat162float(__float2bfloat16_rn(v[c]));
+  store_state_row_bf16(hi_base, r, v);
+  store_state_row_bf16(lo_base, r, lo);
+}
+
+// Hash-backward partial sums of one token over the 128 sketch rows of half HALF.
+// dp[r] = dP of row HALF*128 + r; lo/hi: corner factors of every table of the row group
+// (table j: lo[8j..8j+7], hi[(R/8)j ..]); Ts[j] = sum_b p_b dP_b, As[j*P + p] = sum over
+// corners with bit p set.
+template <int P, int HALF>
+__device__ __forceinline__ void hash_bwd_half(const float* dp, const float* lo, const float* hi,
+                                              float* Ts, float* As) {
+  constexpr int R = 1 << P;
+  constexpr int NHI = R / 8;
+#pragma unroll
+  for (int g8 = 0; g8 < 16; ++g8) {
+    const int row0 = HALF * 128 + g8 * 8;
+    const int j = row0 / R;              // table
+    const int c = (row0 % R) / 8;        // high corner index within the table
+    float m[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = lo[8 * j + e] * dp[g8 * 8 + e];
+    const float z = ((m[0] + m[1]) + (m[2] + m[3])) + ((m[4] + m[5]) + (m[6] + m[7]));
+    const float hz = hi[NHI * j + c];
+    Ts[j] = fmaf(hz, z, Ts[j]);
+    As[j * P + 0] = fmaf(hz, (m[1] + m[3]) + (m[5] + m[7]), As[j * P + 0]);
+    As[j * P + 1] = fmaf(hz, (m[2] + m[3]) + (m[6] + m[7]), As[j * P + 1]);
+    As[j * P + 2] = fmaf(hz, (m[4] + m[5]) + (m[6] + m[7]), As[j * P + 2]);
+    const float w = hz * z;
+#pragma unroll
+    for (int p = 3; p < P; ++p)
+      if ((c >> (p - 3)) & 1) As[j * P + p] += w;
+  }
+}
+
+template <int P, int MODE, bool REV>
+__global__ void __launch_bounds__(kBwThreads, 1)
+    k_bwd_phi(const __grid_constant__ CUtensorMap txa, const __grid_constant__ CUtensorMap txb,
+              const __grid_constant__ CUtensorMap tfa, const __grid_constant__ CUtensorMap tfb,
+              const float* __restrict__ ea, const float* __restrict__ eb,
+              const float* __restrict__ W, const float* __restrict__ init,
+              float* __restrict__ seg_out, float* __restrict__ du_out, Params prm) {
+  constexpr bool HAS_A = MODE != kBuild;      // corner gradients of side a
+  constexpr bool HAS_B = MODE != kReadout;    // state built from side b
+  constexpr bool CAUSAL = MODE == kSweep;
+  constexpr int R = 1 << P;
+  constexpr int TABLES = 256 / R;
+  constexpr int NP = ((TABLES * P + 15) / 16) * 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BwSmem::bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kbCOUNT);
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x, rg = blockIdx.y, h = blockIdx.z;
+  const int64_t s0 = (int64_t)g * prm.seg_len;
+  const int64_t s1 = min64(prm.N, s0 + prm.seg_len);
+  const int nchunks = (int)((s1 - s0 + kC - 1) / kC);
+  const int l0 = rg * TABLES;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kbCOUNT; ++i) mbar_init(bar + i, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x < kAlu) {
+    // projection operand [K = 64 dims][N = NP], W split into bf16 hi + lo
+    for (int e = threadIdx.x; e < 64 * NP; e += kAlu) {
+      const int n = e / 64, kd = e % 64;
+      float w = 0.f;
+      if (n < TABLES * P) w = W[((size_t)(l0 + n / P) * 64 + kd) * P + (n % P)];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+      const uint32_t off = (n >> 3) * 1024 + (kd >> 3) * 128 + (n & 7) * 16 + (kd & 7) * 2;
+      *reinterpret_cast<__nv_bfloat16*>(sm + BwSmem::whi + off) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(sm + BwSmem::wlo + off) = lo;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- initial state: TMEM accumulators (HAS_B) and/or the bf16 copy (HAS_A)
+  const float* init_cta = init + (((size_t)h * prm.n_rg + rg) * prm.G + g) * (size_t)256 * kNV;
+  if (threadIdx.x < kAlu) {
+    const int t = threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    for (int mt = 0; mt < 2; ++mt) {
+      float vals[kNV];
+#pragma unroll
+      for (int c = 0; c < kNV; ++c)
+        vals[c] = prm.have_init ? init_cta[(size_t)(mt * 128 + t) * kNV + c] : 0.f;
+      if (HAS_B) {
+        uint32_t r[16];
+#pragma unroll
+        for (int b = 0; b < 5; ++b) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(vals[b * 16 + e]);
+          tmem_st16(tmem + lane_off + (mt ? BwTm::S1 : BwTm::S0) + b * 16, r);
+        }
+      }
+      if (HAS_A) store_state_row_split(sb + BwSmem::sbf, sb + BwSmem::sbl, mt * 128 + t, vals);
+    }
+    if (HAS_B) tmem_st_wait();
+    fence_proxy_async();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == 4) {
+    // ================================================================ issuer
+    if (lane == 0) {
+      if (HAS_A) { prefetch_tmap(&txa); prefetch_tmap(&tfa); }
+      if (HAS_B) { prefetch_tmap(&txb); prefetch_tmap(&tfb); }
+      const uint32_t id_proj = idesc_bf16(128, NP, 0, 0);
+      const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);   // X Y^T and X S^T
+      const uint32_t id_d3 = idesc_bf16(128, 128, 0, 1);    // A tmem, B MN-major
+      const uint32_t id_up = idesc_bf16(128, kNV, 1, 1);    // A, B MN-major
+      bool ok = true;
+      auto wait = [&](int b, uint32_t par) {
+        if (ok && !mbar_wait(bar + b, par)) { ok = false; s_abort = 1; }
+        return ok;
+      };
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const int c = REV ? nchunks - 1 - i : i;
+        const int t0 = (int)(s0 + (int64_t)c * kC);
+        mbar_arrive_expect_tx(bar + kbTMA, (HAS_A ? 32768u : 0u) + (HAS_B ? 32768u : 0u));
+        if (HAS_A) {
+          tma_load_3d(sm + BwSmem::xa, &txa, 0, t0, h, bar + kbTMA);
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+            tma_load_3d(sm + BwSmem::fa + a * 4096, &tfa, a * 16, t0, h, bar + kbTMA);
+        }
+        if (HAS_B) {
+          tma_load_3d(sm + BwSmem::xb, &txb, 0, t0, h, bar + kbTMA);
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+            tma_load_3d(sm + BwSmem::fb + a * 4096, &tfb, a * 16, t0, h, bar + kbTMA);
+        }
+        if (!wait(kbTMA, i & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint64_t bh = sdesc(sb + BwSmem::whi + s * 256, 128, 1024, kSwizzleNone);
+          const uint64_t bl = sdesc(sb + BwSmem::wlo + s * 256, 128, 1024, kSwizzleNone);
+          if (HAS_A) {
+            const uint64_t a = sdesc(sb + BwSmem::xa + s * 32, 16, 1024, kSwizzle128B);
+            umma_ss(tmem + BwTm::pa, a, bh, id_proj, s > 0);
+            umma_ss(tmem + BwTm::pa, a, bl, id_proj, 1);
+          }
+          if (HAS_B) {
+            const uint64_t a = sdesc(sb + BwSmem::xb + s * 32, 16, 1024, kSwizzle128B);
+            umma_ss(tmem + BwTm::pb, a, bh, id_proj, s > 0);
+            umma_ss(tmem + BwTm::pb, a, bl, id_proj, 1);
+          }
+        }
+        umma_commit(bar + kbPROJ);
+        if (!wait(kbPHI, i & 1)) break;
+        tc_fence_after();
+        if (CAUSAL) {
+          // X Y^T: rows of side a x tokens of side b, K = 80 feature columns
+#pragma unroll
+          for (int s = 0; s < 5; ++s)
+            umma_ss(tmem + BwTm::dw, sdesc(sb + BwSmem::fa + s * 4096, 16, 256, kSwizzle32B),
+                    sdesc(sb + BwSmem::fb + s * 4096, 16, 256, kSwizzle32B), id_128, s > 0);
+          umma_commit(bar + kbDW);
+          if (!wait(kbINTRA, i & 1)) break;
+          tc_fence_after();
+        }
+        if (HAS_A) {
+          for (int half = 0; half < 2 && ok; ++half) {
+            // X S^T over sketch rows half*128 .. +127 (K = 80)
+#pragma unroll
+            for (int s = 0; s < 5; ++s) {
+              const uint64_t xd = sdesc(sb + BwSmem::fa + s * 4096, 16, 256, kSwizzle32B);
+              umma_ss(tmem + BwTm::dp, xd,
+                      sdesc(sb + BwSmem::sbf + half * 20480 + s * 256, 128, 1280, kSwizzleNone),
+                      id_128, s > 0);
+              umma_ss(tmem + BwTm::dp, xd,
+                      sdesc(sb + BwSmem::sbl + half * 20480 + s * 256, 128, 1280, kSwizzleNone),
+                      id_128, 1);
+            }
+            if (CAUSAL) {
+              // + mask(X Y^T) p(b): K = 128 tokens of side b
+#pragma unroll
+              for (int s = 0; s < 8; ++s)
+                umma_ts(tmem + BwTm::dp, tmem + BwTm::intra + s * 8,
+                        sdesc(sb + BwSmem::phb + half * 2048 + s * 8192, 4096, 128, kSwizzleNone),
+                        id_d3, 1);
+            }
+            umma_commit(bar + kbDP);
+            // the next chunk's first half waits for FREE, which follows the release of
+            // this chunk's second half
+            if (half == 0) {
+              if (!wait(kbDPFREE, 0)) break;
+              tc_fence_after();
+            }
+          }
+          if (!ok) break;
+        }
+        if (HAS_B) {
+          // S += p(b)^T Y, both halves of the sketch rows (K = 128 tokens)
+          for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+              umma_ss(tmem + (half ? BwTm::S1 : BwTm::S0),
+                      sdesc(sb + BwSmem::phb + half * 2048 + s * 8192, 4096, 128, kSwizzleNone),
+                      sdesc(sb + BwSmem::fb + s * 512, 4096, 256, kSwizzle32B), id_up, 1);
+          umma_commit(bar + kbUP);
+        }
+        if (!wait(kbFREE, i & 1)) break;
+      }
+    }
+  } else if (warp < 4) {
+    // ================================================================ CUDA-core warps
+    const int t = threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int LP = prm.L * P;
+    for (int i = 0; i < nchunks; ++i) {
+      if (s_abort) break;
+      const int c = REV ? nchunks - 1 - i : i;
+      const int64_t t0 = s0 + (int64_t)c * kC;
+      const bool valid = (t0 + t) < s1;
+      if (!mbar_wait(bar + kbPROJ, i & 1)) { s_abort = 1; break; }
+      tc_fence_after();
+      float ua[NP], ub[NP];
+      uint32_t r[16];
+      float inv_a = 0.f;
+      if (HAS_A) {
+#pragma unroll
+        for (int b = 0; b < NP / 16; ++b) {
+          tmem_ld16(tmem + lane_off + BwTm::pa + b * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ua[b * 16 + e] = __uint_as_float(r[e]);
+        }
+        inv_a = row_inv_norm(sm + BwSmem::xa, t);
+        store_extra_cols(sb + BwSmem::fa, t, ea, (size_t)h * prm.N + t0 + t, valid);
+      }
+      if (HAS_B) {
+#pragma unroll
+        for (int b = 0; b < NP / 16; ++b) {
+          tmem_ld16(tmem + lane_off + BwTm::pb + b * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ub[b * 16 + e] = __uint_as_float(r[e]);
+        }
+        const float sc = row_inv_norm(sm + BwSmem::xb, t) * prm.two_over_tau;
+        write_phi_rows<P>(sb + BwSmem::phb, t, 256, TABLES, ub, sc, valid);
+        store_extra_cols(sb + BwSmem::fb, t, eb, (size_t)h * prm.N + t0 + t, valid);
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      named_bar(1, kAlu);
+      if (t == 0) mbar_arrive(bar + kbPHI);
+
+      if (CAUSAL) {
+        // mask X Y^T (b tokens j <= t, or j >= t in the reverse sweep), round to bf16
+        if (!mbar_wait(bar + kbDW, i & 1)) { s_abort = 1; break; }
+        tc_fence_after();
+        uint32_t packed[64];
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          uint32_t x[64];
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb) tmem_ld16(tmem + lane_off + BwTm::dw + hb * 64 + cb * 16, x + cb * 16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j0 = hb * 64 + 2 * e;
+            const bool k0 = REV ? (j0 >= t) : (j0 <= t);
+            const bool k1 = REV ? (j0 + 1 >= t) : (j0 + 1 <= t);
+            packed[hb * 32 + e] = pack_bf16(k0 ? __uint_as_float(x[2 * e]) : 0.f,
+                                            k1 ? __uint_as_float(x[2 * e + 1]) : 0.f);
+          }
+        }
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) tmem_st16(tmem + lane_off + BwTm::intra + cb * 16, packed + cb * 16);
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar(1, kAlu);
+        if (t == 0) mbar_arrive(bar + kbINTRA);
+      }
+
+      if (HAS_A) {
+        // ---- soft hash backward of side a
+        float sp[TABLES * P], lo[TABLES * 8], hi[TABLES * (R / 8)];
+        const float sc = inv_a * prm.two_over_tau;
+#pragma unroll
+        for (int j = 0; j < TABLES; ++j) {
+          float spj[P], smj[P];
+#pragma unroll
+          for (int p = 0; p < P; ++p) {
+            logistic_fast(ua[j * P + p] * sc, spj[p], smj[p]);
+            sp[j * P + p] = spj[p];
+          }
+#pragma unroll
+          for (int b = 0; b < 8; ++b)
+            lo[8 * j + b] = ((b & 1) ? spj[0] : smj[0]) * ((b & 2) ? spj[1] : smj[1]) *
+                            ((b & 4) ? spj[2] : smj[2]);
+          float hj[R / 8];
+          hj[0] = 1.f;
+          kron_tree<3, P>(hj, spj, smj);
+#pragma unroll
+          for (int cc = 0; cc < R / 8; ++cc) hi[(R / 8) * j + cc] = hj[cc];
+        }
+        float Ts[TABLES], As[TABLES * P];
+#pragma unroll
+        for (int j = 0; j < TABLES; ++j) Ts[j] = 0.f;
+#pragma unroll
+        for (int e = 0; e < TABLES * P; ++e) As[e] = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(bar + kbDP, half)) { s_abort = 1; break; }
+          tc_fence_after();
+          float dp[128];
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            uint32_t x[64];
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tmem + lane_off + BwTm::dp + hb * 64 + cb * 16, x + cb * 16);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 64; ++e) dp[hb * 64 + e] = __uint_as_float(x[e]);
+          }
+          tc_fence_before();
+          named_bar(1, kAlu);
+          if (t == 0) mbar_arrive(bar + kbDPFREE);
+          if (half == 0) hash_bwd_half<P, 0>(dp, lo, hi, Ts, As);
+          else hash_bwd_half<P, 1>(dp, lo, hi, Ts, As);
+        }
+        if (s_abort) break;
+        if (valid) {
+          float* dst = du_out + ((size_t)h * prm.N + t0 + t) * LP + (size_t)l0 * P;
+#pragma unroll
+          for (int j = 0; j < TABLES; ++j)
+#pragma unroll
+            for (int p = 0; p < P; ++p)
+              dst[j * P + p] = prm.two_over_tau * (As[j * P + p] - sp[j * P + p] * Ts[j]);
+        }
+      }
+
+      if (HAS_B) {
+        if (!mbar_wait(bar + kbUP, i & 1)) { s_abort = 1; break; }
+        tc_fence_after();
+        if (CAUSAL) {
+          for (int mt = 0; mt < 2; ++mt) {
+            float vals[kNV];
+            tmem_ld80(tmem + lane_off + (mt ? BwTm::S1 : BwTm::S0), vals);
+            store_state_row_split(sb + BwSmem::sbf, sb + BwSmem::sbl, mt * 128 + t, vals);
+          }
+          fence_proxy_async();
+        }
+      }
+      tc_fence_before();
+      named_bar(1, kAlu);
+      if (t == 0) mbar_arrive(bar + kbFREE);
+    }
+    if (MODE == kBuild && !s_abort) {
+      float* out = seg_out + (((size_t)h * prm.n_rg + rg) * prm.G + g) * (size_t)256 * kNV;
+      for (int mt = 0; mt < 2; ++mt) {
+        float vals[kNV];
+        tmem_ld80(tmem + lane_off + (mt ? BwTm::S1 : BwTm::S0), vals);
+        float4* o4 = reinterpret_cast<float4*>(out + (size_t)(mt * 128 + t) * kNV);
+#pragma unroll
+        for (int cc = 0; cc < kNV / 4; ++cc)
+          o4[cc] = make_float4(vals[4 * cc], vals[4 * cc + 1], vals[4 * cc + 2], vals[4 * cc + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------------------------- helpers
+// g''_i in bf16 (first 64 columns) and its last column -(g_i . o_i)/den'_i in float32.
+// den' comes from the caller's saved den (times L) or from forward accumulators.
+template <typename T, typename TO>
+__global__ void k_bwd_prep(const T* __restrict__ dout, const TO* __restrict__ out,
+                           const float* __restrict__ num, const float* __restrict__ den_in,
+                           __nv_bfloat16* __restrict__ gh, float* __restrict__ gdot,
+                           int64_t rows, float L) {
+  const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= rows) return;
+  const float den = den_in ? den_in[i] * L : num[i * kNumStride + kD];
+  const float inv = 1.0f / den;
+  const float g0 = to_f(dout[i * kD + 2 * lane]), g1 = to_f(dout[i * kD + 2 * lane + 1]);
+  const float o0 = to_f(out[i * kD + 2 * lane]), o1 = to_f(out[i * kD + 2 * lane + 1]);
+  // -(g . o)/den' from the rounded g/den', so that dw_ij = g''_i . [v_j ; 1] is exactly
+  // sum_c bf16(g_c/den') (v_jc - o_ic): no cancellation error when v_j is close to o_i
+  const __nv_bfloat162 r = __floats2bfloat162_rn(g0 * inv, g1 * inv);
+  const float2 rf = __bfloat1622float2(r);
+  const float c = simt::warp_sum(rf.x * o0 + rf.y * o1);
+  reinterpret_cast<__nv_bfloat162*>(gh + i * kD)[lane] = r;
+  if (lane == 0) gdot[i] = -c;
+}
+
+// dst[h][N-1-n] = src[h][n] for 64-wide bf16 rows.
+__global__ void k_reverse_rows(const __nv_bfloat16* __restrict__ src,
+                               __nv_bfloat16* __restrict__ dst, int64_t N, int H) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // one 16-byte piece
+  if (e >= (int64_t)H * N * 8) return;
+  const int64_t row = e >> 3;
+  const int piece = (int)(e & 7);
+  const int64_t h = row / N, n = row % N;
+  const uint4* s = reinterpret_cast<const uint4*>(src + row * kD) + piece;
+  uint4* d = reinterpret_cast<uint4*>(dst + (h * N + (N - 1 - n)) * kD) + piece;
+  *d = *s;
+}
+
+// dv[h][n] = first 64 accumulators of row n (reversed rows: N-1-n) of the anti-causal
+// sweep.
+template <typename T>
+__global__ void k_dv_out(const float* __restrict__ num, T* __restrict__ dv, int64_t N, int H,
+                         int reversed) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)H * N * kD) return;
+  const int64_t row = e / kD;
+  const int c = (int)(e % kD);
+  const int64_t h = row / N, n = row % N;
+  const int64_t src = reversed ? h * N + (N - 1 - n) : row;
+  dv[e] = from_f<T>(num[src * kNumStride + c]);
+}
+
+// dx from du: dxhat = sum_{l,p} W[l][:][p] du[l*P + p]; dx = (dxhat - xhat (xhat . dxhat))
+// / |x| (dxhat / eps when |x| <= eps).  Also per-block partial sums of
+// dW[l][:][p] = sum_n xhat_n du_n[l*P + p] into part[block][L*P][64].
+// 256 threads, 64 tokens per tile; LP = L*P <= kMaxLP.
+constexpr int kMaxLP = 256;
+constexpr int kFinTok = 64;
+template <typename T>
+__global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
+                                                     const float* __restrict__ du,
+                                                     const float* __restrict__ W,
+                                                     T* __restrict__ dx, float* __restrict__ part,
+                                                     int64_t rows, int L, int P) {
+  extern __shared__ float fsm[];
+  const int LP = L * P;
+  const int ldu = LP + 1;
+  float* Wt = fsm;                       // [LP][64]
+  float* dus = Wt + LP * 64;             // [64 tokens][LP + 1]
+  float* xh = dus + kFinTok * ldu;       // [64 tokens][65]
+  const int tid = threadIdx.x;
+  for (int e = tid; e < LP * 64; e += 256) {
+    const int lp = e / 64, d = e % 64;
+    const int l = lp / P, p = lp % P;
+    Wt[e] = W[((size_t)l * 64 + d) * P + p];
+  }
+  // dW accumulators: dims 4*(tid%16)..+3, rows lp = tid/16 + 16m
+  float acc[kMaxLP / 16][4];
+#pragma unroll
+  for (int m = 0; m < kMaxLP / 16; ++m)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
+  const int tok = tid >> 2, qd = (tid & 3) * 16;
+  const int dq4 = (tid & 15) * 4, lpg = tid >> 4;
+  for (int64_t base = (int64_t)blockIdx.x * kFinTok; base < rows;
+       base += (int64_t)gridDim.x * kFinTok) {
+    __syncthreads();
+    const int ntok = (int)min64(kFinTok, rows - base);
+    for (int e = tid; e < kFinTok * LP; e += 256) {
+      const int tt = e / LP, lp = e % LP;
+      dus[tt * ldu + lp] = tt < ntok ? du[(base + tt) * LP + lp] : 0.f;
+    }
+    __syncthreads();
+    // ---- dx: 4 threads per token, 16 dims each
+    const bool live = tok < ntok;
+    float xv[16], dxh[16];
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      xv[e] = live ? to_f(x[(base + tok) * kD + qd + e]) : 0.f;
+      ss = fmaf(xv[e], xv[e], ss);
+      dxh[e] = 0.f;
+    }
+    for (int lp = 0; lp < LP; ++lp) {
+      const float u = dus[tok * ldu + lp];
+      const float4* w4 = reinterpret_cast<const float4*>(Wt + lp * 64 + qd);
+#pragma unroll
+      for (int e4 = 0; e4 < 4; ++e4) {
+        const float4 w = w4[e4];
+        dxh[4 * e4] = fmaf(w.x, u, dxh[4 * e4]);
+        dxh[4 * e4 + 1] = fmaf(w.y, u, dxh[4 * e4 + 1]);
+        dxh[4 * e4 + 2] = fmaf(w.z, u, dxh[4 * e4 + 2]);
+        dxh[4 * e4 + 3] = fmaf(w.w, u, dxh[4 * e4 + 3]);
+      }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float n = sqrtf(ss);
+    const float inv = 1.0f / fmaxf(n, kEpsNorm);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dot = fmaf(xv[e] * inv, dxh[e], dot);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    if (live) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float xhat = xv[e] * inv;
+        const float g = n > kEpsNorm ? (dxh[e] - xhat * dot) * inv : dxh[e] / kEpsNorm;
+        dx[(base + tok) * kD + qd + e] = from_f<T>(g);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) xh[tok * 65 + qd + e] = xv[e] * inv;
+    __syncthreads();
+    // ---- dW partials
+    for (int tt = 0; tt < ntok; ++tt) {
+      const float x0 = xh[tt * 65 + dq4], x1 = xh[tt * 65 + dq4 + 1];
+      const float x2 = xh[tt * 65 + dq4 + 2], x3 = xh[tt * 65 + dq4 + 3];
+#pragma unroll
+      for (int m = 0; m < kMaxLP / 16; ++m) {
+        const int lp = lpg + 16 * m;
+        if (lp < LP) {
+          const float u = dus[tt * ldu + lp];
+          acc[m][0] = fmaf(x0, u, acc[m][0]);
+          acc[m][1] = fmaf(x1, u, acc[m][1]);
+          acc[m][2] = fmaf(x2, u, acc[m][2]);
+          acc[m][3] = fmaf(x3, u, acc[m][3]);
+        }
+      }
+    }
+  }
+  float* o = part + (size_t)blockIdx.x * LP * 64;
+#pragma unroll
+  for (int m = 0; m < kMaxLP / 16; ++m) {
+    const int lp = lpg + 16 * m;
+    if (lp < LP)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[lp * 64 + dq4 + e] = acc[m][e];
+  }
+}
+
+inline size_t finalize_smem(int LP) {
+  return ((size_t)LP * 64 + (size_t)kFinTok * (LP + 1) + (size_t)kFinTok * 65) * sizeof(float);
+}
+
+// dW[l][d][p] = sum of the partials of both sides, in fixed order.
+__global__ void k_bwd_dw_reduce(const float* __restrict__ pq, const float* __restrict__ pk,
+                                int nblocks, float* __restrict__ dW, int L, int P) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // over L*64*P, W layout
+  if (e >= L * 64 * P) return;
+  const int l = e / (64 * P), d = (e / P) % 64, p = e % P;
+  const int LP = L * P;
+  const size_t off = (size_t)(l * P + p) * 64 + d;
+  float acc = 0.f;
+  for (int b = 0; b < nblocks; ++b) acc += pq[(size_t)b * LP * 64 + off];
+  for (int b = 0; b < nblocks; ++b) acc += pk[(size_t)b * LP * 64 + off];
+  dW[e] = acc;
+}
+
+// 3-D view [H][N][64] bf16 of a feature tensor for the 32B-swizzled loads: boxes of
+// 16 columns x 128 rows.
+inline bool encode_feat_tmap(CUtensorMap* m, const void* base, int64_t N, int H) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)H};
+  cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+  cuuint32_t box[3] = {16, (cuuint32_t)kC, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+}  // namespace race
