@@ -223,10 +223,15 @@ __global__ void __launch_bounds__(kS8Threads, 1)
 
   if (warp == 12) {
     // ================================================================ issuer
-    if (lane == 0) {
-      prefetch_tmap(&tq);
-      prefetch_tmap(&tk);
-      prefetch_tmap(&tv);
+    // The whole warp runs this loop (waits included); TMA copies, MMAs and commits are
+    // issued by one elected lane (the same lane every time).
+    {
+      if (elect_one()) {
+        prefetch_tmap(&tq);
+        prefetch_tmap(&tk);
+        prefetch_tmap(&tv);
+      }
+      __syncwarp();
       const uint32_t id_proj = idesc_bf16(128, 16, 0, 0);
       const uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
       const uint32_t id_ro = idesc_bf16(128, kNV, 0, 1);   // A tmem (K-major), B MN-major
@@ -247,36 +252,46 @@ __global__ void __launch_bounds__(kS8Threads, 1)
       const float* inv_q = inv_norms + (size_t)h * inv_stride;
       const float* inv_k = inv_norms + ((size_t)prm.H + h) * inv_stride;
       bool ok = true;
-      auto wait = [&](int b, uint32_t par) {
+      auto wait = [&](int b, uint32_t par) {   // warp-uniform outcome
         if (ok && !mbar_wait(bar + b, par)) ok = false;
+        ok = __all_sync(0xffffffffu, ok);
         return ok;
       };
       auto load_qk = [&](int c) {
         const int st = c & 1;
         const int t0 = (int)(s0 + (int64_t)c * kC);
-        mbar_arrive_expect_tx(bar + k8_QKFULL0 + st, 32768 + 1024);
-        tma_load_3d(sm + (st ? S8Smem::q1 : S8Smem::q0), &tq, 0, t0, h, bar + k8_QKFULL0 + st);
-        tma_load_3d(sm + (st ? S8Smem::k1 : S8Smem::k0), &tk, 0, t0, h, bar + k8_QKFULL0 + st);
-        uint8_t* inv = sm + (st ? S8Smem::inv1 : S8Smem::inv0);
-        bulk_load(inv, inv_q + t0, 512, bar + k8_QKFULL0 + st);
-        bulk_load(inv + 512, inv_k + t0, 512, bar + k8_QKFULL0 + st);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar + k8_QKFULL0 + st, 32768 + 1024);
+          tma_load_3d(sm + (st ? S8Smem::q1 : S8Smem::q0), &tq, 0, t0, h, bar + k8_QKFULL0 + st);
+          tma_load_3d(sm + (st ? S8Smem::k1 : S8Smem::k0), &tk, 0, t0, h, bar + k8_QKFULL0 + st);
+          uint8_t* inv = sm + (st ? S8Smem::inv1 : S8Smem::inv0);
+          bulk_load(inv, inv_q + t0, 512, bar + k8_QKFULL0 + st);
+          bulk_load(inv + 512, inv_k + t0, 512, bar + k8_QKFULL0 + st);
+        }
+        __syncwarp();
       };
       auto load_v = [&](int c) {
         const int st = c & 1;
         const int t0 = (int)(s0 + (int64_t)c * kC);
-        mbar_arrive_expect_tx(bar + k8_VFULL0 + st, 16384);
-        tma_load_3d(sm + (st ? S8Smem::v1 : S8Smem::v0), &tv, 0, t0, h, bar + k8_VFULL0 + st);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar + k8_VFULL0 + st, 16384);
+          tma_load_3d(sm + (st ? S8Smem::v1 : S8Smem::v0), &tv, 0, t0, h, bar + k8_VFULL0 + st);
+        }
+        __syncwarp();
       };
       auto issue_proj = [&](int c) {
         const int st = c & 1;
         const uint64_t dq = sdesc(sb + (st ? S8Smem::q1 : S8Smem::q0), 16, 1024, kSwizzle128B);
         const uint64_t dk = sdesc(sb + (st ? S8Smem::k1 : S8Smem::k0), 16, 1024, kSwizzle128B);
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          umma_ss(tmem + S8Tm::pq, dq + 2 * s, d_w + 16 * s, id_proj, s > 0);
-          umma_ss(tmem + S8Tm::pk, dk + 2 * s, d_w + 16 * s, id_proj, s > 0);
+          for (int s = 0; s < 4; ++s) {
+            umma_ss(tmem + S8Tm::pq, dq + 2 * s, d_w + 16 * s, id_proj, s > 0);
+            umma_ss(tmem + S8Tm::pk, dk + 2 * s, d_w + 16 * s, id_proj, s > 0);
+          }
+          umma_commit(bar + k8_PROJ);
         }
-        umma_commit(bar + k8_PROJ);
+        __syncwarp();
       };
       if (nchunks > 0) {
         load_qk(0);
@@ -304,33 +319,45 @@ __global__ void __launch_bounds__(kS8Threads, 1)
         if (!wait(k8_PHQ, par) || !wait(k8_PHK0, par)) break;
         SW_TRACE(c, 1);
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ts(tmem + S8Tm::qk, tmem + S8Tm::phq + s * 8,
-                  d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, s > 0);
+          for (int s = 0; s < 8; ++s)
+            umma_ts(tmem + S8Tm::qk, tmem + S8Tm::phq + s * 8,
+                    d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, s > 0);
+        }
+        __syncwarp();
         if (!wait(k8_SBF0, par) || !wait(k8_SBF1, par)) break;
         if (c > 0 && !wait(k8_NUMFREE, par ^ 1)) break;
         SW_TRACE(c, 2);
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 16; ++s)
-          umma_ts(tmem + S8Tm::num, tmem + S8Tm::phq + s * 8, d_ro + 32 * s, id_ro, s > 0);
+          for (int s = 0; s < 16; ++s)
+            umma_ts(tmem + S8Tm::num, tmem + S8Tm::phq + s * 8, d_ro + 32 * s, id_ro, s > 0);
+        }
+        __syncwarp();
         if (!wait(k8_VFULL0 + st, spar)) break;
         SW_TRACE(c, 3);
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ss(tmem + S8Tm::S0, d_up0 + 128 * s, d_vone + vstep * s, id_up, 1);
-        umma_commit(bar + k8_HALF0);
+          for (int s = 0; s < 8; ++s)
+            umma_ss(tmem + S8Tm::S0, d_up0 + 128 * s, d_vone + vstep * s, id_up, 1);
+          umma_commit(bar + k8_HALF0);
+        }
+        __syncwarp();
         // ---- half 1
         if (!wait(k8_PHK1, par)) break;
         SW_TRACE(c, 4);
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 8; s < 16; ++s)
-          umma_ts(tmem + S8Tm::qk, tmem + S8Tm::phq + s * 8,
-                  d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, 1);
-        umma_commit(bar + k8_QKDONE);      // QK complete; p(q) of this chunk no longer read
+          for (int s = 8; s < 16; ++s)
+            umma_ts(tmem + S8Tm::qk, tmem + S8Tm::phq + s * 8,
+                    d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, 1);
+          umma_commit(bar + k8_QKDONE);    // QK complete; p(q) of this chunk no longer read
+        }
+        __syncwarp();
         // next chunk's projections go into the p(q) columns just released (in issue
         // order after the last MMA that reads p(q) of this chunk)
         if (c + 1 < nchunks) {
@@ -338,20 +365,26 @@ __global__ void __launch_bounds__(kS8Threads, 1)
           tc_fence_after();
           issue_proj(c + 1);
         }
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ss(tmem + S8Tm::S1, d_up1 + 128 * s, d_vone + vstep * s, id_up, 1);
-        umma_commit(bar + k8_HALF1);
+          for (int s = 0; s < 8; ++s)
+            umma_ss(tmem + S8Tm::S1, d_up1 + 128 * s, d_vone + vstep * s, id_up, 1);
+          umma_commit(bar + k8_HALF1);
+        }
+        __syncwarp();
         // ---- masked in-chunk weights are ready in tensor memory
         if (!wait(k8_CONV, par)) break;
         SW_TRACE(c, 5);
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ts(tmem + S8Tm::num,
-                  tmem + (s < 4 ? S8Tm::intraA + s * 8 : S8Tm::intraB + (s - 4) * 8),
-                  d_vone + vstep * s, id_ro, 1);
-        umma_commit(bar + k8_AV);
+          for (int s = 0; s < 8; ++s)
+            umma_ts(tmem + S8Tm::num,
+                    tmem + (s < 4 ? S8Tm::intraA + s * 8 : S8Tm::intraB + (s - 4) * 8),
+                    d_vone + vstep * s, id_ro, 1);
+          umma_commit(bar + k8_AV);
+        }
+        __syncwarp();
         if (c + 2 < nchunks) {       // v tile of stage st: AV was its last reader
           if (!wait(k8_AV, par)) break;
           SW_TRACE(c, 7);
