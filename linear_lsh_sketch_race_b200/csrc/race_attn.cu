@@ -14,7 +14,7 @@
 #include "tc_kernels.cuh"
 #include "tc_ptx.cuh"
 #include "tc_sweep.cuh"
-#include "tc_sweep256.cuh"
+#include "tc_sweep_pipe.cuh"
 #include "tc_backward.cuh"
 
 namespace race {
@@ -379,10 +379,10 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
   if (mode == tc::kSweep && P == 8 && prm.rows == 256 && inv_norms) {
     CUtensorMap tnum;
     if (!tc::encode_num_tmap(&tnum, num, prm.N, prm.H)) return RACE_ERR_CUDA;
-    RACE_CU(set_smem(tc::k_sweep256, tc::S8Smem::alloc));
+    RACE_CU(set_smem(tc::k_sweep_pipe, tc::SPSmem::alloc));
     RACE_LAUNCH("tc_causal_sweep", s);
-    tc::k_sweep256<<<grid, tc::kS8Threads, tc::S8Smem::alloc, s>>>(
-        tq, tk, tv, W, init, inv_norms, inv_stride, tnum, prm);
+    tc::k_sweep_pipe<<<grid, tc::kSPThreads, tc::SPSmem::alloc, s>>>(
+        tq, tk, tv, W, init, inv_norms, inv_stride, tnum, num, prm);
   } else if (mode == tc::kSweep && prm.rows == 256) {
     constexpr int TABLES = 256 >> P;
     RACE_CU(set_smem(tc::k_sweep<P, TABLES>, tc::SwSmem::alloc));
