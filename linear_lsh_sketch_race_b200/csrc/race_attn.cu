@@ -566,6 +566,38 @@ race_status_t bw_dispatch(int P, int mode, bool rev, const tc::Params& prm,
   return RACE_ERR_UNSUPPORTED;
 }
 
+template <int MT>
+race_status_t finalize_launch_mt(const __nv_bfloat16* q, const float* duq, const float* W,
+                                 __nv_bfloat16* dq, float* partq, const __nv_bfloat16* k,
+                                 const float* duk, __nv_bfloat16* dk, float* partk,
+                                 int64_t rows, int L, int P, int blocks, size_t fsm,
+                                 cudaStream_t s) {
+  RACE_CU(set_smem(tc::k_bwd_finalize<__nv_bfloat16, MT>, fsm));
+  RACE_LAUNCH("tc_bwd_finalize", s);
+  tc::k_bwd_finalize<__nv_bfloat16, MT><<<blocks, 256, fsm, s>>>(q, duq, W, dq, partq, rows, L, P);
+  tc::k_bwd_finalize<__nv_bfloat16, MT><<<blocks, 256, fsm, s>>>(k, duk, W, dk, partk, rows, L, P);
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+// dq, dk and the dW partials for L*P projections (MT = ceil(L*P / 16) <= 16).
+race_status_t finalize_launch(int mt, const __nv_bfloat16* q, const float* duq, const float* W,
+                              __nv_bfloat16* dq, float* partq, const __nv_bfloat16* k,
+                              const float* duk, __nv_bfloat16* dk, float* partk, int64_t rows,
+                              int L, int P, int blocks, size_t fsm, cudaStream_t s) {
+#define RACE_FIN(M)                                                                      \
+  case M:                                                                                \
+    return finalize_launch_mt<M>(q, duq, W, dq, partq, k, duk, dk, partk, rows, L, P, \
+                                 blocks, fsm, s)
+  switch (mt) {
+    RACE_FIN(1); RACE_FIN(2); RACE_FIN(3); RACE_FIN(4); RACE_FIN(5); RACE_FIN(6); RACE_FIN(7);
+    RACE_FIN(8); RACE_FIN(9); RACE_FIN(10); RACE_FIN(11); RACE_FIN(12); RACE_FIN(13);
+    RACE_FIN(14); RACE_FIN(15); RACE_FIN(16);
+  }
+#undef RACE_FIN
+  return RACE_ERR_UNSUPPORTED;
+}
+
 template <typename TO>
 race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __nv_bfloat16* k,
                           const __nv_bfloat16* v, const float* W, const TO* out,
@@ -666,15 +698,9 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   RACE_CU(cudaGetLastError());
   // ---- dq, dk through the projections and the normalisation; dW
   const size_t fsm = tc::finalize_smem(LP);
-  RACE_CU(set_smem(tc::k_bwd_finalize<__nv_bfloat16>, fsm));
-  {
-    RACE_LAUNCH("tc_bwd_finalize", s);
-    tc::k_bwd_finalize<__nv_bfloat16><<<pl.fin_blocks, 256, fsm, s>>>(q, duq, W, dq, partq,
-                                                                       rows, a->L, a->P);
-    tc::k_bwd_finalize<__nv_bfloat16><<<pl.fin_blocks, 256, fsm, s>>>(k, duk, W, dk, partk,
-                                                                       rows, a->L, a->P);
-  }
-  RACE_CU(cudaGetLastError());
+  st = finalize_launch(tc::finalize_mt(LP), q, duq, W, dq, partq, k, duk, dk, partk, rows, a->L,
+                       a->P, pl.fin_blocks, fsm, s);
+  if (st != RACE_OK) return st;
   const int nW = a->L * kD * a->P;
   {
     RACE_LAUNCH("tc_bwd_dW_reduce", s);

@@ -211,21 +211,28 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 
   if (warp == 4) {
     // ================================================================ issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (waits included, with a warp-uniform outcome); TMA
+    // copies, MMAs and commits are issued by one elected lane (the same one every time).
+    if (elect_one()) {
       if (HAS_A) { prefetch_tmap(&txa); prefetch_tmap(&tfa); }
       if (HAS_B) { prefetch_tmap(&txb); prefetch_tmap(&tfb); }
-      const uint32_t id_proj = idesc_bf16(128, NP, 0, 0);
-      const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);   // X Y^T and X S^T
-      const uint32_t id_d3 = idesc_bf16(128, 128, 0, 1);    // A tmem, B MN-major
-      const uint32_t id_up = idesc_bf16(128, kNV, 1, 1);    // A, B MN-major
-      bool ok = true;
-      auto wait = [&](int b, uint32_t par) {
-        if (ok && !mbar_wait(bar + b, par)) { ok = false; s_abort = 1; }
-        return ok;
-      };
-      for (int i = 0; i < nchunks && ok; ++i) {
-        const int c = REV ? nchunks - 1 - i : i;
-        const int t0 = (int)(s0 + (int64_t)c * kC);
+    }
+    __syncwarp();
+    const uint32_t id_proj = idesc_bf16(128, NP, 0, 0);
+    const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);   // X Y^T and X S^T
+    const uint32_t id_d3 = idesc_bf16(128, 128, 0, 1);    // A tmem, B MN-major
+    const uint32_t id_up = idesc_bf16(128, kNV, 1, 1);    // A, B MN-major
+    bool ok = true;
+    auto wait = [&](int b, uint32_t par) {
+      if (ok && !mbar_wait(bar + b, par)) ok = false;
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok && lane == 0) s_abort = 1;
+      return ok;
+    };
+    for (int i = 0; i < nchunks && ok; ++i) {
+      const int c = REV ? nchunks - 1 - i : i;
+      const int t0 = (int)(s0 + (int64_t)c * kC);
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar + kbTMA, (HAS_A ? 32768u : 0u) + (HAS_B ? 32768u : 0u));
         if (HAS_A) {
           tma_load_3d(sm + BwSmem::xa, &txa, 0, t0, h, bar + kbTMA);
@@ -239,8 +246,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           for (int a = 0; a < 4; ++a)
             tma_load_3d(sm + BwSmem::fb + a * 4096, &tfb, a * 16, t0, h, bar + kbTMA);
         }
-        if (!wait(kbTMA, i & 1)) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      if (!wait(kbTMA, i & 1)) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const uint64_t bh = sdesc(sb + BwSmem::whi + s * 256, 128, 1024, kSwizzleNone);
@@ -257,20 +267,26 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           }
         }
         umma_commit(bar + kbPROJ);
-        if (!wait(kbPHI, i & 1)) break;
-        tc_fence_after();
-        if (CAUSAL) {
-          // X Y^T: rows of side a x tokens of side b, K = 80 feature columns
+      }
+      __syncwarp();
+      if (!wait(kbPHI, i & 1)) break;
+      tc_fence_after();
+      if (CAUSAL) {
+        // X Y^T: rows of side a x tokens of side b, K = 80 feature columns
+        if (elect_one()) {
 #pragma unroll
           for (int s = 0; s < 5; ++s)
             umma_ss(tmem + BwTm::dw, sdesc(sb + BwSmem::fa + s * 4096, 16, 256, kSwizzle32B),
                     sdesc(sb + BwSmem::fb + s * 4096, 16, 256, kSwizzle32B), id_128, s > 0);
           umma_commit(bar + kbDW);
-          if (!wait(kbINTRA, i & 1)) break;
-          tc_fence_after();
         }
-        if (HAS_A) {
-          for (int half = 0; half < 2 && ok; ++half) {
+        __syncwarp();
+        if (!wait(kbINTRA, i & 1)) break;
+        tc_fence_after();
+      }
+      if (HAS_A) {
+        for (int half = 0; half < 2 && ok; ++half) {
+          if (elect_one()) {
             // X S^T over sketch rows half*128 .. +127 (K = 80)
 #pragma unroll
             for (int s = 0; s < 5; ++s) {
@@ -291,17 +307,20 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                         id_d3, 1);
             }
             umma_commit(bar + kbDP);
-            // the next chunk's first half waits for FREE, which follows the release of
-            // this chunk's second half
-            if (half == 0) {
-              if (!wait(kbDPFREE, 0)) break;
-              tc_fence_after();
-            }
           }
-          if (!ok) break;
+          __syncwarp();
+          // the next chunk's first half waits for FREE, which follows the release of
+          // this chunk's second half
+          if (half == 0) {
+            if (!wait(kbDPFREE, 0)) break;
+            tc_fence_after();
+          }
         }
-        if (HAS_B) {
-          // S += p(b)^T Y, both halves of the sketch rows (K = 128 tokens)
+        if (!ok) break;
+      }
+      if (HAS_B) {
+        // S += p(b)^T Y, both halves of the sketch rows (K = 128 tokens)
+        if (elect_one()) {
           for (int half = 0; half < 2; ++half)
 #pragma unroll
             for (int s = 0; s < 8; ++s)
@@ -310,8 +329,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                       sdesc(sb + BwSmem::fb + s * 512, 4096, 256, kSwizzle32B), id_up, 1);
           umma_commit(bar + kbUP);
         }
-        if (!wait(kbFREE, i & 1)) break;
+        __syncwarp();
       }
+      if (!wait(kbFREE, i & 1)) break;
     }
   } else if (warp < 4) {
     // ================================================================ CUDA-core warps
@@ -532,115 +552,149 @@ __global__ void k_dv_out(const float* __restrict__ num, T* __restrict__ dv, int6
 // dx from du: dxhat = sum_{l,p} W[l][:][p] du[l*P + p]; dx = (dxhat - xhat (xhat . dxhat))
 // / |x| (dxhat / eps when |x| <= eps).  Also per-block partial sums of
 // dW[l][:][p] = sum_n xhat_n du_n[l*P + p] into part[block][L*P][64].
-// 256 threads, 64 tokens per tile; LP = L*P <= kMaxLP.
+// Hash backward, last steps, per token x (a row of q or k) with du = dL/du over the L*P
+// projections: dx^ = W du (projection transpose), dx = (dx^ - x^ (x^ . dx^)) / |x|
+// (normalisation Jacobian), and dW partials x^ du^T summed over the tokens of each block.
+// 256 threads, 64 tokens per tile, LP padded to LPP = 16 * MT with zero columns.
+// Register tiles: dx^ as 4 tokens x 4 dims per thread over K = LPP in steps of 4; dW as
+// MT consecutive rows x 4 dims per thread over the 64 tokens of the tile.
 constexpr int kMaxLP = 256;
 constexpr int kFinTok = 64;
-template <typename T>
+template <typename T, int MT>
 __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
                                                      const float* __restrict__ du,
                                                      const float* __restrict__ W,
                                                      T* __restrict__ dx, float* __restrict__ part,
                                                      int64_t rows, int L, int P) {
-  extern __shared__ float fsm[];
+  constexpr int LPP = 16 * MT;
+  constexpr int LDS = LPP + 4;          // row stride of the du tile (16-byte aligned rows)
+  extern __shared__ float4 fsm4[];
+  float* fsm = reinterpret_cast<float*>(fsm4);
   const int LP = L * P;
-  const int ldu = LP + 1;
-  float* Wt = fsm;                       // [LP][64]
-  float* dus = Wt + LP * 64;             // [64 tokens][LP + 1]
-  float* xh = dus + kFinTok * ldu;       // [64 tokens][65]
+  float* Wt = fsm;                       // [LPP][64]: row lp = plane p of table l
+  float* dus = Wt + LPP * 64;            // [64 tokens][LDS]
+  float* xh = dus + kFinTok * LDS;       // [64 tokens][68]: x / |x|
+  float* ninv = xh + kFinTok * 68;       // [64]: 1 / max(|x|, eps), 0 for padding rows
   const int tid = threadIdx.x;
-  for (int e = tid; e < LP * 64; e += 256) {
+  for (int e = tid; e < LPP * 64; e += 256) {
     const int lp = e / 64, d = e % 64;
-    const int l = lp / P, p = lp % P;
-    Wt[e] = W[((size_t)l * 64 + d) * P + p];
+    Wt[e] = lp < LP ? W[((size_t)(lp / P) * 64 + d) * P + (lp % P)] : 0.f;
   }
-  // dW accumulators: dims 4*(tid%16)..+3, rows lp = tid/16 + 16m
-  float acc[kMaxLP / 16][4];
+  const int tg = tid >> 4, dg = (tid & 15) * 4;   // dx^: tokens tg + 16 i, dims dg..dg+3
+  const int rg = (tid >> 4) * MT;                 // dW: rows rg..rg+MT-1, dims dg..dg+3
+  float acc[MT][4];
 #pragma unroll
-  for (int m = 0; m < kMaxLP / 16; ++m)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[m][e] = 0.f;
-  const int tok = tid >> 2, qd = (tid & 3) * 16;
-  const int dq4 = (tid & 15) * 4, lpg = tid >> 4;
   for (int64_t base = (int64_t)blockIdx.x * kFinTok; base < rows;
        base += (int64_t)gridDim.x * kFinTok) {
     __syncthreads();
     const int ntok = (int)min64(kFinTok, rows - base);
-    for (int e = tid; e < kFinTok * LP; e += 256) {
-      const int tt = e / LP, lp = e % LP;
-      dus[tt * ldu + lp] = tt < ntok ? du[(base + tt) * LP + lp] : 0.f;
+    for (int e = tid; e < kFinTok * LPP; e += 256) {
+      const int tt = e / LPP, lp = e % LPP;
+      dus[tt * LDS + lp] = (tt < ntok && lp < LP) ? du[(base + tt) * LP + lp] : 0.f;
     }
-    __syncthreads();
-    // ---- dx: 4 threads per token, 16 dims each
-    const bool live = tok < ntok;
-    float xv[16], dxh[16];
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      xv[e] = live ? to_f(x[(base + tok) * kD + qd + e]) : 0.f;
-      ss = fmaf(xv[e], xv[e], ss);
-      dxh[e] = 0.f;
-    }
-    for (int lp = 0; lp < LP; ++lp) {
-      const float u = dus[tok * ldu + lp];
-      const float4* w4 = reinterpret_cast<const float4*>(Wt + lp * 64 + qd);
-#pragma unroll
-      for (int e4 = 0; e4 < 4; ++e4) {
-        const float4 w = w4[e4];
-        dxh[4 * e4] = fmaf(w.x, u, dxh[4 * e4]);
-        dxh[4 * e4 + 1] = fmaf(w.y, u, dxh[4 * e4 + 1]);
-        dxh[4 * e4 + 2] = fmaf(w.z, u, dxh[4 * e4 + 2]);
-        dxh[4 * e4 + 3] = fmaf(w.w, u, dxh[4 * e4 + 3]);
-      }
-    }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    const float n = sqrtf(ss);
-    const float inv = 1.0f / fmaxf(n, kEpsNorm);
-    float dot = 0.f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) dot = fmaf(xv[e] * inv, dxh[e], dot);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-    if (live) {
+    {   // x / |x|: 4 threads per token, 16 dims each
+      const int tok = tid >> 2, qd = (tid & 3) * 16;
+      const bool live = tok < ntok;
+      float xv[16], ss = 0.f;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float xhat = xv[e] * inv;
-        const float g = n > kEpsNorm ? (dxh[e] - xhat * dot) * inv : dxh[e] / kEpsNorm;
-        dx[(base + tok) * kD + qd + e] = from_f<T>(g);
+        xv[e] = live ? to_f(x[(base + tok) * kD + qd + e]) : 0.f;
+        ss = fmaf(xv[e], xv[e], ss);
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      const float inv = 1.0f / fmaxf(sqrtf(ss), kEpsNorm);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) xh[tok * 68 + qd + e] = xv[e] * inv;
+      if ((tid & 3) == 0) ninv[tok] = live ? inv : 0.f;
+    }
+    __syncthreads();
+    // ---- dx^ = W du for tokens tg + 16 i
+    float dxh[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dxh[i][e] = 0.f;
+#pragma unroll 2
+    for (int k = 0; k < LPP; k += 4) {
+      float4 w[4], u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const float4*>(Wt + (k + j) * 64 + dg);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const float4*>(dus + (tg + 16 * i) * LDS + k);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float uu[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          dxh[i][0] = fmaf(w[j].x, uu[j], dxh[i][0]);
+          dxh[i][1] = fmaf(w[j].y, uu[j], dxh[i][1]);
+          dxh[i][2] = fmaf(w[j].z, uu[j], dxh[i][2]);
+          dxh[i][3] = fmaf(w[j].w, uu[j], dxh[i][3]);
+        }
       }
     }
+    // ---- dx = (dx^ - x^ (x^ . dx^)) / |x|; the 16 threads of a token are 16 lanes
 #pragma unroll
-    for (int e = 0; e < 16; ++e) xh[tok * 65 + qd + e] = xv[e] * inv;
-    __syncthreads();
-    // ---- dW partials
-    for (int tt = 0; tt < ntok; ++tt) {
-      const float x0 = xh[tt * 65 + dq4], x1 = xh[tt * 65 + dq4 + 1];
-      const float x2 = xh[tt * 65 + dq4 + 2], x3 = xh[tt * 65 + dq4 + 3];
+    for (int i = 0; i < 4; ++i) {
+      const int tok = tg + 16 * i;
+      const float4 xv = *reinterpret_cast<const float4*>(xh + tok * 68 + dg);
+      float dot = xv.x * dxh[i][0] + xv.y * dxh[i][1] + xv.z * dxh[i][2] + xv.w * dxh[i][3];
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 8);
+      const float inv = ninv[tok];
+      if (tok < ntok) {
+        T* o = dx + (base + tok) * kD + dg;
+        o[0] = from_f<T>((dxh[i][0] - xv.x * dot) * inv);
+        o[1] = from_f<T>((dxh[i][1] - xv.y * dot) * inv);
+        o[2] = from_f<T>((dxh[i][2] - xv.z * dot) * inv);
+        o[3] = from_f<T>((dxh[i][3] - xv.w * dot) * inv);
+      }
+    }
+    // ---- dW partials: rows rg..rg+MT-1 (table l, plane p), dims dg..dg+3
+#pragma unroll 2
+    for (int tt = 0; tt < kFinTok; ++tt) {
+      const float4 xv = *reinterpret_cast<const float4*>(xh + tt * 68 + dg);
+      float u[MT];
 #pragma unroll
-      for (int m = 0; m < kMaxLP / 16; ++m) {
-        const int lp = lpg + 16 * m;
-        if (lp < LP) {
-          const float u = dus[tt * ldu + lp];
-          acc[m][0] = fmaf(x0, u, acc[m][0]);
-          acc[m][1] = fmaf(x1, u, acc[m][1]);
-          acc[m][2] = fmaf(x2, u, acc[m][2]);
-          acc[m][3] = fmaf(x3, u, acc[m][3]);
+      for (int m = 0; m < MT; m += 4) {
+        if (m + 4 <= MT) {
+          const float4 u4 = *reinterpret_cast<const float4*>(dus + tt * LDS + rg + m);
+          u[m] = u4.x; u[m + 1] = u4.y; u[m + 2] = u4.z; u[m + 3] = u4.w;
+        } else {
+#pragma unroll
+          for (int mm = m; mm < MT; ++mm) u[mm] = dus[tt * LDS + rg + mm];
         }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        acc[m][0] = fmaf(xv.x, u[m], acc[m][0]);
+        acc[m][1] = fmaf(xv.y, u[m], acc[m][1]);
+        acc[m][2] = fmaf(xv.z, u[m], acc[m][2]);
+        acc[m][3] = fmaf(xv.w, u[m], acc[m][3]);
       }
     }
   }
   float* o = part + (size_t)blockIdx.x * LP * 64;
 #pragma unroll
-  for (int m = 0; m < kMaxLP / 16; ++m) {
-    const int lp = lpg + 16 * m;
+  for (int m = 0; m < MT; ++m) {
+    const int lp = rg + m;
     if (lp < LP)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[lp * 64 + dq4 + e] = acc[m][e];
+      for (int e = 0; e < 4; ++e) o[lp * 64 + dg + e] = acc[m][e];
   }
 }
 
+inline int finalize_mt(int LP) { return (LP + 15) / 16; }
 inline size_t finalize_smem(int LP) {
-  return ((size_t)LP * 64 + (size_t)kFinTok * (LP + 1) + (size_t)kFinTok * 65) * sizeof(float);
+  const int LPP = 16 * finalize_mt(LP);
+  return ((size_t)LPP * 64 + (size_t)kFinTok * (LPP + 4) + (size_t)kFinTok * 68 + kFinTok) *
+         sizeof(float);
 }
 
 // dW[l][d][p] = sum of the partials of both sides, in fixed order.
