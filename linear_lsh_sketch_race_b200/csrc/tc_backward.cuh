@@ -100,6 +100,40 @@ __device__ __forceinline__ void store_state_row_split(uint32_t hi_base, uint32_t
 // dp[r] = dP of row HALF*128 + r; lo/hi: corner factors of every table of the row group
 // (table j: lo[8j..8j+7], hi[(R/8)j ..]); Ts[j] = sum_b p_b dP_b, As[j*P + p] = sum over
 // corners with bit p set.
+// write_phi_rows for 256 sketch rows with the loop over groups of four high corners kept
+// rolled (a smaller instruction footprint for the sweep's CUDA-core warps): corner
+// c = 4g + jj has high factor p34[jj] (planes 3-4) times the product over planes 5.. chosen
+// by the bits of g.
+template <int P, int TABLES>
+__device__ __forceinline__ void write_phi_rows_rolled(uint32_t tile, int t, const float* u,
+                                                      float scale, bool valid) {
+  constexpr int R = 1 << P;
+  constexpr int NG = R / 32;
+  const uint32_t base = tile + (t >> 3) * (256 * 16) + (t & 7) * 16;
+#pragma unroll
+  for (int j = 0; j < TABLES; ++j) {
+    float sp[P], sm[P];
+#pragma unroll
+    for (int p = 0; p < P; ++p) logistic_fast(u[j * P + p] * scale, sp[p], sm[p]);
+    float lo[8], p34[4];
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+      lo[b] = ((b & 1) ? sp[0] : sm[0]) * ((b & 2) ? sp[1] : sm[1]) * ((b & 4) ? sp[2] : sm[2]);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      p34[jj] = (valid ? 1.f : 0.f) * ((jj & 1) ? sp[3] : sm[3]) * ((jj & 2) ? sp[4] : sm[4]);
+#pragma unroll 1
+    for (int g = 0; g < NG; ++g) {
+      float hg = 1.f;
+#pragma unroll
+      for (int p = 5; p < P; ++p) hg *= ((g >> (p - 5)) & 1) ? sp[p] : sm[p];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        store_chunk(base + (uint32_t)((j * R) / 8 + 4 * g + jj) * 128, hg * p34[jj], lo);
+    }
+  }
+}
+
 template <int P, int HALF>
 __device__ __forceinline__ void hash_bwd_half(const float* dp, const float* lo, const float* hi,
                                               float* Ts, float* As) {
@@ -368,7 +402,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           for (int e = 0; e < 16; ++e) ub[b * 16 + e] = __uint_as_float(r[e]);
         }
         const float sc = row_inv_norm(sm + BwSmem::xb, t) * prm.two_over_tau;
-        write_phi_rows<P>(sb + BwSmem::phb, t, 256, TABLES, ub, sc, valid);
+        write_phi_rows_rolled<P, TABLES>(sb + BwSmem::phb, t, ub, sc, valid);
         store_extra_cols(sb + BwSmem::fb, t, eb, (size_t)h * prm.N + t0 + t, valid);
       }
       fence_proxy_async();
@@ -380,24 +414,25 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         // mask X Y^T (b tokens j <= t, or j >= t in the reverse sweep), round to bf16
         if (!mbar_wait(bar + kbDW, i & 1)) { s_abort = 1; break; }
         tc_fence_after();
-        uint32_t packed[64];
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          uint32_t x[64];
-#pragma unroll
-          for (int cb = 0; cb < 4; ++cb) tmem_ld16(tmem + lane_off + BwTm::dw + hb * 64 + cb * 16, x + cb * 16);
+        // key block kb (32 keys): loaded, masked and rounded before the next block's
+        // load; the bf16 pairs of block kb land in columns intra + 16 kb, which hold fp32
+        // keys already loaded (the first 64 fp32 columns)
+#pragma unroll 1
+        for (int kb = 0; kb < 4; ++kb) {
+          uint32_t x[32], o[16];
+          tmem_ld16(tmem + lane_off + BwTm::dw + kb * 32, x);
+          tmem_ld16(tmem + lane_off + BwTm::dw + kb * 32 + 16, x + 16);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j0 = hb * 64 + 2 * e;
+          for (int e = 0; e < 16; ++e) {
+            const int j0 = kb * 32 + 2 * e;
             const bool k0 = REV ? (j0 >= t) : (j0 <= t);
             const bool k1 = REV ? (j0 + 1 >= t) : (j0 + 1 <= t);
-            packed[hb * 32 + e] = pack_bf16(k0 ? __uint_as_float(x[2 * e]) : 0.f,
-                                            k1 ? __uint_as_float(x[2 * e + 1]) : 0.f);
+            o[e] = pack_bf16(k0 ? __uint_as_float(x[2 * e]) : 0.f,
+                             k1 ? __uint_as_float(x[2 * e + 1]) : 0.f);
           }
+          tmem_st16(tmem + lane_off + BwTm::intra + kb * 16, o);
         }
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) tmem_st16(tmem + lane_off + BwTm::intra + cb * 16, packed + cb * 16);
         tmem_st_wait();
         tc_fence_before();
         named_bar(1, kAlu);
@@ -466,6 +501,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         if (!mbar_wait(bar + kbUP, i & 1)) { s_abort = 1; break; }
         tc_fence_after();
         if (CAUSAL) {
+#pragma unroll 1
           for (int mt = 0; mt < 2; ++mt) {
             float vals[kNV];
             tmem_ld80(tmem + lane_off + (mt ? BwTm::S1 : BwTm::S0), vals);
