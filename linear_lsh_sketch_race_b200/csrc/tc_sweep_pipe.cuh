@@ -100,7 +100,32 @@ struct Corners {
   float lo[8];
   float p34[4];
   float f5[2], f6[2], f7[2];
+  uint64_t lo2[4];   // float pairs (lo[2e], lo[2e+1]) in one 64-bit register
 };
+
+// bf16 pair (h * lo2.x, h * lo2.y): one packed float multiply and one packed conversion,
+// the same roundings as two float multiplies and a conversion.
+__device__ __forceinline__ uint32_t mul_pack_bf16(uint64_t lo2, uint64_t hh) {
+  uint32_t out;
+  asm("{\n\t.reg .b64 pr;\n\t.reg .f32 a, b;\n\t"
+      "mul.rn.f32x2 pr, %1, %2;\n\t"
+      "mov.b64 {a, b}, pr;\n\t"
+      "cvt.rn.bf16x2.f32 %0, b, a;\n\t}"
+      : "=r"(out)
+      : "l"(lo2), "l"(hh));
+  return out;
+}
+__device__ __forceinline__ uint64_t bcast_f32x2(float h) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(h));
+  return r;
+}
+__device__ __forceinline__ uint64_t pair_f32x2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 __device__ __forceinline__ void corners_of(const float* sp, const float* sm, float valid,
                                            Corners& k) {
 #pragma unroll
@@ -111,6 +136,8 @@ __device__ __forceinline__ void corners_of(const float* sp, const float* sm, flo
   k.f5[0] = sm[5]; k.f5[1] = sp[5];
   k.f6[0] = sm[6]; k.f6[1] = sp[6];
   k.f7[0] = sm[7]; k.f7[1] = sp[7];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) k.lo2[e] = pair_f32x2(k.lo[2 * e], k.lo[2 * e + 1]);
 }
 __device__ __forceinline__ float corners_h5(const Corners& k, int g) {
   return ((g & 1) ? k.f5[1] : k.f5[0]) * ((g & 2) ? k.f6[1] : k.f6[0]) *
@@ -397,10 +424,9 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         uint32_t v16[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float hv = h5 * k.p34[j];
+          const uint64_t hh = bcast_f32x2(h5 * k.p34[j]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            v16[j * 4 + e] = pack_bf16(hv * k.lo[2 * e], hv * k.lo[2 * e + 1]);
+          for (int e = 0; e < 4; ++e) v16[j * 4 + e] = mul_pack_bf16(k.lo2[e], hh);
         }
         tmem_st16(tmem + lane_off + SPTm::pq + 16 * g, v16);
         if ((g & 3) == 3) {        // a bucket half is complete
@@ -452,8 +478,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         for (int gg = 0; gg < 4; ++gg) {
           const float h5 = corners_h5(k, 4 * half + gg);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            store_chunk(phk_addr(base, t, 4 * gg + j), h5 * k.p34[j], k.lo);
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t hh = bcast_f32x2(h5 * k.p34[j]);
+            st_shared_v4(phk_addr(base, t, 4 * gg + j), mul_pack_bf16(k.lo2[0], hh),
+                         mul_pack_bf16(k.lo2[1], hh), mul_pack_bf16(k.lo2[2], hh),
+                         mul_pack_bf16(k.lo2[3], hh));
+          }
         }
         fence_proxy_async();
         __syncwarp();
