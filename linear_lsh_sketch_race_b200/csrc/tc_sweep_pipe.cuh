@@ -62,12 +62,6 @@ struct SPTm {
   static constexpr uint32_t S0 = 0, S1 = 80, num = 160, qk = 240, pq = 368, proj = 496;
 };
 
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
 
 // bf16 copy of the 80-column state row held in tensor-memory lane (this thread) at
 // column `col`, as row r of the 32B-swizzled readout operand (see store_state_row_sw32).
