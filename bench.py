@@ -86,6 +86,31 @@ def kernel_work(name: str, wl: I.Workload):
     return table[name] * th
 
 
+def rank_heads(rank: int, heads_per_rank: int):
+    """Global head indices of one rank: heads are independent (W is shared), so with weak
+    scaling rank r owns heads r*H .. r*H + H - 1 of the global batch of heads."""
+    return [rank * heads_per_rank + h for h in range(heads_per_rank)]
+
+
+def allreduce_dw(dW, world: int):
+    """dW is a sum over all heads and tokens: the per-rank partial sums are added with one
+    all-reduce (NCCL on GPUs; any backend of the default process group)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(dW, op=dist.ReduceOp.SUM)
+    return dW
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Step time of the job = the slowest rank's device time."""
+    if world <= 1:
+        return ms
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples while the timed region runs."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -208,7 +233,7 @@ def run_ours(args, wl: I.Workload):
                                 device_id=dev)
     ra.load()
     backward = not args.fwd_only
-    heads = [rank * wl.H + h for h in range(wl.H)]
+    heads = rank_heads(rank, wl.H)
     x = I.make_inputs(wl, dev, heads=heads, with_dout=backward)
     q, k, v, W = x["q"], x["k"], x["v"], x["W"]
     dout = x.get("dout")
@@ -232,8 +257,7 @@ def run_ours(args, wl: I.Workload):
         ra.race_forward_ex(q, k, v, W, out, a, stream)
         if backward:
             ra.race_backward_ex(q, k, v, W, out, dout, dq, dk, dv, dW, a, stream)
-            if world > 1:
-                dist.all_reduce(dW)
+            allreduce_dw(dW, world)
 
     def timed(fn, n):
         if world > 1:
@@ -248,12 +272,7 @@ def run_ours(args, wl: I.Workload):
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        ms = e0.elapsed_time(e1) / n
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = t.item()
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -361,8 +380,7 @@ def run_e2e(args, wl, x, a, ra, dev, stream, world, backward):
             if backward:
                 ra.race_backward_ex(dev_in["q"], dev_in["k"], dev_in["v"], W, out,
                                     dev_in["dout"], *grads, a, stream)
-                if world > 1:
-                    dist.all_reduce(grads[3])
+                allreduce_dw(grads[3], world)
             for t, h in zip(outs, host_out):
                 h.copy_(t, non_blocking=True)
 
@@ -378,11 +396,7 @@ def run_e2e(args, wl, x, a, ra, dev, stream, world, backward):
             step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / n
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = t.item()
+        ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
         tokens = wl.batch * wl.N * world
         return {"value": tokens / (ms / 1000), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
