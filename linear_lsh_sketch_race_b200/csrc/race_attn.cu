@@ -238,6 +238,22 @@ race_status_t simt_forward_num(const SimtPlan& p, const T* q, const T* k, const 
   return RACE_OK;
 }
 
+// o = num / den: the vector kernel when the output rows are 16-byte aligned (the
+// workspace always is), else one thread per output.
+template <typename TO>
+void launch_normalize(const float* num, TO* out, float* den, int64_t rows, float inv_L,
+                      cudaStream_t s) {
+  if ((reinterpret_cast<uintptr_t>(out) & 15) == 0) {
+    const int64_t n8 = rows * (kD / 8);
+    const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, (int64_t)kPlanSMs * 16);
+    simt::k_normalize8<TO><<<(unsigned)std::max<int64_t>(blocks, 1), 256, 0, s>>>(
+        num, out, den, rows, inv_L);
+  } else {
+    simt::k_normalize<TO><<<(unsigned)((rows + 3) / 4), 256, 0, s>>>(num, out, den, rows,
+                                                                      inv_L);
+  }
+}
+
 template <typename T, typename TO>
 race_status_t simt_forward(const race_args_t* a, const T* q, const T* k, const T* v,
                            const float* W, TO* out, char* ws, cudaStream_t s) {
@@ -247,8 +263,7 @@ race_status_t simt_forward(const race_args_t* a, const T* q, const T* k, const T
   const int64_t rows = (int64_t)a->H * a->N;
   {
     RACE_LAUNCH("simt_normalize", s);
-    simt::k_normalize<TO><<<(unsigned)((rows + 3) / 4), 256, 0, s>>>(
-        reinterpret_cast<float*>(ws + p.off_num), out, a->den, rows, 1.f / a->L);
+    launch_normalize(reinterpret_cast<float*>(ws + p.off_num), out, a->den, rows, 1.f / a->L, s);
   }
   RACE_CU(cudaGetLastError());
   return RACE_OK;
@@ -441,7 +456,7 @@ race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k,
   if (a->causal && pl.P == 8 && prm.rows == 256) {
     inv_norms = reinterpret_cast<float*>(ws + pl.off_inv);
     RACE_LAUNCH("tc_inv_norms", s);
-    tc::k_inv_norms<<<dim3((unsigned)((a->N + 255) / 256), 2 * a->H), 256, 0, s>>>(
+    tc::k_inv_norms<<<dim3((unsigned)((a->N + 127) / 128), 2 * a->H), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), inv_norms,
         a->N, a->H, pl.inv_stride);
   }
@@ -462,8 +477,7 @@ race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, con
   const int64_t rows = (int64_t)a->H * a->N;
   {
     RACE_LAUNCH("tc_normalize", s);
-    simt::k_normalize<TO><<<(unsigned)((rows + 3) / 4), 256, 0, s>>>(num, out, a->den, rows,
-                                                                      1.f / a->L);
+    launch_normalize(num, out, a->den, rows, 1.f / a->L, s);
   }
   RACE_CU(cudaGetLastError());
   return RACE_OK;

@@ -306,6 +306,42 @@ __global__ void k_normalize(const float* __restrict__ num, TO* __restrict__ out,
   if (den_out && c == 0) den_out[i] = den * inv_L;
 }
 
+// Eight consecutive outputs of a row, 16-byte aligned destination.
+__device__ __forceinline__ void store8(float* dst, const float* v) {
+  __stcs(reinterpret_cast<float4*>(dst), make_float4(v[0], v[1], v[2], v[3]));
+  __stcs(reinterpret_cast<float4*>(dst) + 1, make_float4(v[4], v[5], v[6], v[7]));
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* dst, const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+    w[e] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  __stcs(reinterpret_cast<uint4*>(dst), make_uint4(w[0], w[1], w[2], w[3]));
+}
+
+// k_normalize with one thread per eight outputs (vector loads and stores, streaming
+// cache hints); num rows and out rows must be 16-byte aligned.  Grid-stride loop.
+template <typename TO>
+__global__ void k_normalize8(const float* __restrict__ num, TO* __restrict__ out,
+                             float* __restrict__ den_out, int64_t rows, float inv_L) {
+  const int64_t n8 = rows * (kD / 8);
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n8;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = g >> 3;
+    const int part = (int)(g & 7);
+    const float* r = num + i * kNumStride;
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(r + part * 8));
+    const float4 b = __ldcs(reinterpret_cast<const float4*>(r + part * 8) + 1);
+    const float den = r[kD];
+    const float o[8] = {a.x / den, a.y / den, a.z / den, a.w / den,
+                        b.x / den, b.y / den, b.z / den, b.w / den};
+    store8(out + i * kD + part * 8, o);
+    if (den_out && part == 0) den_out[i] = den * inv_L;
+  }
+}
+
 // --------------------------------------------------------------------------- //
 // backward
 // g''_i = [g_i / den'_i , -(g_i . o_i) / den'_i]  with den' = L * den.

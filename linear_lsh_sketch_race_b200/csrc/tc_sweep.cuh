@@ -34,9 +34,27 @@ __device__ unsigned long long g_sweep_trace[kTraceChunks * kTraceEvents];
     if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (c) < kTraceChunks)    \
       g_sweep_trace[(c) * kTraceEvents + (ev)] = clock64();                              \
   } while (0)
+// Per-CTA record in row = linear CTA index: 25 SM id, 26/27 global timer at start/end,
+// 38/39 clock64 at start/end.
+__device__ __forceinline__ void sw_trace_cta(bool end) {
+  const int row = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  if (threadIdx.x != 0 || row >= kTraceChunks) return;
+  unsigned long long gt;
+  unsigned int sm;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+  unsigned long long* r = g_sweep_trace + row * kTraceEvents;
+  r[end ? 27 : 26] = gt;
+  r[end ? 39 : 38] = clock64();
+  r[25] = sm;
+}
+#define SW_TRACE_CTA(end) sw_trace_cta(end)
 #else
 #define SW_TRACE(c, ev) \
   do {                  \
+  } while (0)
+#define SW_TRACE_CTA(end) \
+  do {                    \
   } while (0)
 #endif
 

@@ -11,29 +11,40 @@ namespace race {
 namespace tc {
 
 // 1/max(|x|, eps) of every row of q and k into out[side][h][stride] (side 0: q, 1: k);
-// grid (ceil(N/256), 2*H).  Entries stride - N .. of each head are never written and
-// never used (they pad the last chunk so it can be bulk-copied whole).
+// grid (ceil(N/128), 2*H), 256 threads: eight threads per row, one 16-byte load each, so
+// a warp reads four whole rows per load; each thread covers four rows 32 apart (four
+// loads in flight).  The squares are summed over the eight lanes of a row with shuffles.
+// Entries stride - N .. of each head are never written and never used (they pad the
+// last chunk so it can be bulk-copied whole).
 __global__ void k_inv_norms(const __nv_bfloat16* __restrict__ q,
                             const __nv_bfloat16* __restrict__ k, float* __restrict__ out,
                             int64_t N, int H, int64_t stride) {
-  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int part = threadIdx.x & 7;
   const int sh = blockIdx.y;                 // side * H + head
-  if (n >= N) return;
   const int side = sh >= H, h = sh - side * H;
-  const __nv_bfloat16* x = (side ? k : q) + ((size_t)h * N + n) * kD;
-  const uint4* r = reinterpret_cast<const uint4*>(x);
-  float s = 0.f;
+  const __nv_bfloat16* x = (side ? k : q) + (size_t)h * N * kD + part * 8;
+  const int64_t n0 = (int64_t)blockIdx.x * 128 + (threadIdx.x >> 3);
+  uint4 w[4];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 w = __ldg(r + c);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  for (int r = 0; r < 4; ++r) {
+    const int64_t n = n0 + 32 * r;
+    w[r] = n < N ? __ldg(reinterpret_cast<const uint4*>(x + n * kD)) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const uint32_t ws[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+    float s = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[e]));
       s = fmaf(f.x, f.x, fmaf(f.y, f.y, s));
     }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    const int64_t n = n0 + 32 * r;
+    if (n < N && part == 0) out[(size_t)sh * stride + n] = 1.0f / fmaxf(sqrtf(s), kEpsNorm);
   }
-  out[(size_t)sh * stride + n] = 1.0f / fmaxf(sqrtf(s), kEpsNorm);
 }
 
 // Expand the 256 corner probabilities of one token: bucket b = 8*c + e has value

@@ -3,23 +3,25 @@
 // workload.  Soft bucketization, bucket aggregation and readout: [JA] §2.1; causal
 // prefix state: [JA] §2.2.
 //
-// Tensor-core order per chunk c (one elected lane of warp 16 issues everything):
+// Tensor-core work of chunk c, in two streams issued by two warps (one elected lane each):
 //
-//   PROJ_K(c+1)  u_k = x_k (W_hi + W_lo)            -> PROJ (16 tensor-memory columns)
-//   QK(c)        p(q) p(k)^T over 256 buckets        -> QK   (A: p(q) in tensor memory)
-//   PROJ_Q(c+1)  u_q                                  -> PROJ
-//   RO(c)        p(q) S_bf16                          -> NUM  (then p(q) is free)
-//   UPD(c)       S_h += p(k)_h^T [v | 1], h = 0, 1    -> S0, S1
-//   AV(c)        mask(QK) [v | 1]                     -> NUM
+//   warp 16: QK(c)        p(q) p(k)^T over 256 buckets   -> QK   (A: p(q) in tensor memory)
+//            RO(c)        p(q) S_bf16                     -> NUM  (then p(q) is free)
+//            AV(c)        mask(QK) [v | 1]                -> NUM
+//   warp 17: PROJ_Q(c+1)  u_q = x_q (W_hi + W_lo)        -> PROJ (16 tensor-memory columns)
+//            UPD(c)       S_h += p(k)_h^T [v | 1], h = 0, 1 -> S0, S1
+//            PROJ_K(c+2)  u_k                             -> PROJ
+//
+// The waits and bookkeeping of one stream are covered by the other's MMAs: the tensor
+// core's queue holds only a few tens of cycles of work ahead of a single issuer.
 //
 // CUDA-core warp groups (one warp per tensor-memory lane quadrant each):
 //   warps 0-3   expand p(q) of chunk c+1 into tensor memory once RO(c) has read p(q);
 //   warps 4-7   expand p(k) of chunk c+1 into one of three 32 KB half-buffers
-//               (bucket halves; a half-buffer is free once the state update that read it
-//               has completed);
+//               (bucket halves; a half-buffer is free once both QK and the state update
+//               that read it have completed);
 //   warps 8-11  mask QK(c) and round it to bf16 in place; bf16 copy of S for RO(c+1);
-//   warps 12-15 move NUM rows to the float32 output accumulators (TMA reduce-add);
-//   warp 16     TMA and tcgen05 issue.
+//   warps 12-15 move NUM rows to the float32 output accumulators (TMA reduce-add).
 // Every producer/consumer pair has its own mbarrier; a producer can be at most one
 // phase ahead of its consumer, so parity waits stay unambiguous.
 #pragma once
@@ -29,13 +31,15 @@
 namespace race {
 namespace tc {
 
-constexpr int kSPThreads = 544;
+constexpr int kSPThreads = 576;
 
 enum SPBar : int {
   sp_QT = 0, sp_KT, sp_VT0, sp_VT1,
   sp_PROJK_FULL, sp_PROJK_READ, sp_PROJQ_FULL, sp_PROJQ_READ,
   sp_PHQ0, sp_PHQ1, sp_PHK0, sp_PHK1, sp_PHK2, sp_KFREE0, sp_KFREE1, sp_KFREE2,
-  sp_QK_FULL, sp_CONV, sp_PQ_FREE, sp_UPD0, sp_UPD1, sp_SBF, sp_AV_DONE, sp_NUMFREE,
+  sp_KFREEA0, sp_KFREEA1, sp_KFREEA2,
+  sp_QK_FULL, sp_CONV, sp_PQ_FREE, sp_UPD0, sp_UPD1, sp_SREAD0, sp_SREAD1, sp_SBF,
+  sp_AV_DONE, sp_NUMFREE, sp_RO_ISSUED,
   sp_COUNT
 };
 
@@ -64,25 +68,35 @@ struct SPTm {
 
 
 // bf16 copy of the 80-column state row held in tensor-memory lane (this thread) at
-// column `col`, as row r of the 32B-swizzled readout operand (see store_state_row_sw32).
-__device__ __forceinline__ void restage_row(uint32_t taddr, uint32_t sbf, int r) {
+// column `col`: two batches of loads (48 + 32 columns), one wait each, packed to 40
+// bf16 pairs.  After this returns the tensor-memory row may be overwritten.
+__device__ __forceinline__ void restage_load(uint32_t taddr, uint32_t* pk) {
+  uint32_t v[48];
+  tmem_ld16(taddr, v);
+  tmem_ld16(taddr + 16, v + 16);
+  tmem_ld16(taddr + 32, v + 32);
+  tmem_ld_wait();
+#pragma unroll
+  for (int e = 0; e < 24; ++e) pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+  tmem_ld16(taddr + 48, v);
+  tmem_ld16(taddr + 64, v + 16);
+  tmem_ld_wait();
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    pk[24 + e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+}
+
+// Row r of the 32B-swizzled readout operand (see store_state_row_sw32) from 40 bf16 pairs.
+__device__ __forceinline__ void restage_store(uint32_t sbf, int r, const uint32_t* pk) {
   const uint32_t rb = sbf + (r >> 3) * 256 + (r & 7) * 32;
   const uint32_t flip = (r >> 2) & 1;
-#pragma unroll 1
-  for (int a = 0; a < 5; ++a) {
-    uint32_t v[16];
-    tmem_ld16(taddr + a * 16, v);
-    tmem_ld_wait();
+#pragma unroll
+  for (int a = 0; a < 5; ++a)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t* x = v + hh * 8;
-      st_shared_v4(rb + a * 8192 + ((hh ^ flip) << 4),
-                   pack_bf16(__uint_as_float(x[0]), __uint_as_float(x[1])),
-                   pack_bf16(__uint_as_float(x[2]), __uint_as_float(x[3])),
-                   pack_bf16(__uint_as_float(x[4]), __uint_as_float(x[5])),
-                   pack_bf16(__uint_as_float(x[6]), __uint_as_float(x[7])));
+      const uint32_t* x = pk + a * 8 + hh * 4;
+      st_shared_v4(rb + a * 8192 + ((hh ^ flip) << 4), x[0], x[1], x[2], x[3]);
     }
-  }
 }
 
 // Corner probabilities of one token in factored form: bucket b = 8c + e, c = 4g + j,
@@ -162,7 +176,8 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     for (int i = 0; i < sp_COUNT; ++i) {
       const bool by_warps = i == sp_PHQ0 ||
                             i == sp_PHQ1 || (i >= sp_PHK0 && i <= sp_PHK2) || i == sp_CONV ||
-                            i == sp_SBF || i == sp_NUMFREE;
+                            i == sp_SBF || i == sp_NUMFREE || i == sp_SREAD0 ||
+                            i == sp_SREAD1;
       mbar_init(bar + i, by_warps ? 4 : 1);
     }
     fence_mbar_init();
@@ -213,6 +228,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   __syncthreads();
   tc_fence_after();
 
+  SW_TRACE_CTA(false);
   bool ok = true;
   // Warp-uniform bounded wait: a timeout anywhere in the warp ends the warp's loop.
   auto wait = [&](int b, uint32_t par) {
@@ -224,7 +240,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 
   // TMA copies: q/k tiles (with their 1/|x|) of chunk x+1 are issued by the q/k side
   // once it has read chunk x's projections (single buffer each); v tiles of chunk x+2 by
-  // the output warps once AV(x) has completed (two stages).  The issuer only issues MMAs.
+  // the masking warps once UPD(x) and AV(x) have completed (two stages).
   const float* inv_q = inv_norms + (size_t)h * inv_stride;
   const float* inv_k = inv_norms + ((size_t)prm.H + h) * inv_stride;
   auto t0_of = [&](int c) { return (int)(s0 + (int64_t)c * kC); };
@@ -247,10 +263,16 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     if (c + 3 < n) tma_prefetch_3d(&tv, 0, t0_of(c + 3), h);
   };
 
-  if (warp == 16) {
-    // ================================================================ issuer
-    // Per chunk c: QK(c) (two bucket halves), RO(c), PROJ_Q(c+1), UPD(c), AV(c),
-    // PROJ_K(c+2).  Each wait is on work that the MMAs queued before it give time for.
+  if (warp >= 16) {
+    // ================================================================ issuers
+    // Two warps issue two independent MMA streams, so that each one's waits and
+    // bookkeeping between issue blocks are covered by the other's MMAs (the MMA queue
+    // holds only a few tens of cycles of work ahead of a single issuer):
+    //   warp 16: QK(c) over the two bucket halves, RO(c), AV(c)       (p(q) side)
+    //   warp 17: PROJ_Q(c+1), UPD(c) over the two halves, PROJ_K(c+2) (state, projections)
+    // A p(k) half-buffer is free once both QK (warp 16) and UPD (warp 17) have read it;
+    // the bf16 state is rewritten only after RO(c) has read it, and UPD(c+1) of a bucket
+    // half starts once that half of the state after chunk c has been read out.
     const uint32_t id_proj = idesc_bf16(128, 16, 0, 0);
     const uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
     const uint32_t id_ro = idesc_bf16(128, kNV, 0, 1);   // A tmem (K-major), B MN-major
@@ -274,111 +296,137 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       }
       __syncwarp();
     };
-    if (n > 0) {
-      if (elect_one()) {
-        prefetch_tmap(&tq);
-        prefetch_tmap(&tk);
-        prefetch_tmap(&tv);
-        for (int c = 1; c < 3 && c < n; ++c) {
-          tma_prefetch_3d(&tq, 0, t0_of(c), h);
-          tma_prefetch_3d(&tk, 0, t0_of(c), h);
-          tma_prefetch_3d(&tv, 0, t0_of(c), h);
+    if (warp == 16) {
+      for (int c = 0; c < n && ok; ++c) {
+        const uint32_t par = c & 1;
+        const int i0 = 2 * c, i1 = 2 * c + 1;
+        const int b0 = i0 % 3, b1 = i1 % 3;
+        const uint32_t m0 = (uint32_t)(i0 / 3), m1 = (uint32_t)(i1 / 3);
+        const uint64_t d_vone = (c & 1) ? d_vone1 : d_vone0;
+        SW_TRACE(c, 0);
+        // ---- in-chunk QK over the two bucket halves
+        if (!wait(sp_PHQ0, par) || !wait(sp_PHK0 + b0, m0 & 1)) break;
+        SW_TRACE(c, 1);
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t d_qk = sdesc(pk_base + b0 * 32768, 16, 1024, kSwizzle128B);
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            umma_ts(tmem + SPTm::qk, tmem + SPTm::pq + s * 8,
+                    d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, s > 0);
+          umma_commit(bar + sp_KFREEA0 + b0);
         }
-        load_k(0);
-        load_q(0);
-        load_v(0);
-        if (n > 1) load_v(1);
-      }
-      __syncwarp();
-      // PROJ holds, in turn, PROJ_K(0), PROJ_Q(0), PROJ_K(1), PROJ_Q(1), ...; each fill
-      // waits until the previous one was read.
-      if (wait(sp_KT, 0)) proj(d_xk, sp_PROJK_FULL);
-      if (wait(sp_PROJK_READ, 0) && wait(sp_QT, 0)) proj(d_xq, sp_PROJQ_FULL);
-      if (n > 1 && wait(sp_PROJQ_READ, 0) && wait(sp_KT, 1)) proj(d_xk, sp_PROJK_FULL);
-    }
-    for (int c = 0; c < n && ok; ++c) {
-      const uint32_t par = c & 1;
-      const int i0 = 2 * c, i1 = 2 * c + 1;
-      const int b0 = i0 % 3, b1 = i1 % 3;
-      const uint32_t m0 = (uint32_t)(i0 / 3), m1 = (uint32_t)(i1 / 3);
-      const uint64_t d_vone = (c & 1) ? d_vone1 : d_vone0;
-      SW_TRACE(c, 0);
-      // ---- in-chunk QK over the two bucket halves
-      if (!wait(sp_PHQ0, par) || !wait(sp_PHK0 + b0, m0 & 1)) break;
-      SW_TRACE(c, 1);
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t d_qk = sdesc(pk_base + b0 * 32768, 16, 1024, kSwizzle128B);
+        __syncwarp();
+        if (!wait(sp_PHQ1, par) || !wait(sp_PHK0 + b1, m1 & 1)) break;
+        SW_TRACE(c, 2);
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t d_qk = sdesc(pk_base + b1 * 32768, 16, 1024, kSwizzle128B);
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ts(tmem + SPTm::qk, tmem + SPTm::pq + s * 8,
-                  d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, s > 0);
-      }
-      __syncwarp();
-      if (!wait(sp_PHQ1, par) || !wait(sp_PHK0 + b1, m1 & 1)) break;
-      SW_TRACE(c, 2);
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t d_qk = sdesc(pk_base + b1 * 32768, 16, 1024, kSwizzle128B);
+          for (int s = 0; s < 8; ++s)
+            umma_ts(tmem + SPTm::qk, tmem + SPTm::pq + 64 + s * 8,
+                    d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, 1);
+          umma_commit(bar + sp_QK_FULL);
+          umma_commit(bar + sp_KFREEA0 + b1);
+        }
+        __syncwarp();
+        // ---- readout against the state before the chunk; then p(q) is free
+        if (c > 0 && (!wait(sp_SBF, (c - 1) & 1) || !wait(sp_NUMFREE, (c - 1) & 1))) break;
+        SW_TRACE(c, 3);
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ts(tmem + SPTm::qk, tmem + SPTm::pq + 64 + s * 8,
-                  d_qk + (uint64_t)((s >> 2) * 1024 + (s & 3) * 2), id_qk, 1);
-        umma_commit(bar + sp_QK_FULL);
-      }
-      __syncwarp();
-      // ---- readout against the state before the chunk; then p(q) is free
-      if (c > 0 && (!wait(sp_SBF, (c - 1) & 1) || !wait(sp_NUMFREE, (c - 1) & 1))) break;
-      SW_TRACE(c, 3);
-      tc_fence_after();
-      if (elect_one()) {
+          for (int s = 0; s < 16; ++s)
+            umma_ts(tmem + SPTm::num, tmem + SPTm::pq + s * 8, d_ro + 32 * s, id_ro, s > 0);
+          umma_commit(bar + sp_PQ_FREE);
+          mbar_arrive(bar + sp_RO_ISSUED);
+        }
+        __syncwarp();
+        SW_TRACE(c, 9);
+        // ---- masked in-chunk weights times [v | 1]
+        if (!wait(sp_CONV, par) || !wait(sp_VT0 + (c & 1), (c >> 1) & 1)) break;
+        SW_TRACE(c, 5);
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < 16; ++s)
-          umma_ts(tmem + SPTm::num, tmem + SPTm::pq + s * 8, d_ro + 32 * s, id_ro, s > 0);
-        umma_commit(bar + sp_PQ_FREE);
+          for (int s = 0; s < 8; ++s)
+            umma_ts(tmem + SPTm::num, tmem + SPTm::qk + s * 8, d_vone + vstep * s, id_ro, 1);
+          umma_commit(bar + sp_AV_DONE);
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      // ---- q projections of chunk c+1
-      if (c + 1 < n) {
-        if (!wait(sp_PROJK_READ, (c + 1) & 1) || !wait(sp_QT, (c + 1) & 1)) break;
-        proj(d_xq, sp_PROJQ_FULL);
+    } else {
+      if (n > 0) {
+        if (elect_one()) {
+          prefetch_tmap(&tq);
+          prefetch_tmap(&tk);
+          prefetch_tmap(&tv);
+          for (int c = 1; c < 3 && c < n; ++c) {
+            tma_prefetch_3d(&tq, 0, t0_of(c), h);
+            tma_prefetch_3d(&tk, 0, t0_of(c), h);
+            tma_prefetch_3d(&tv, 0, t0_of(c), h);
+          }
+          load_k(0);
+          load_q(0);
+          load_v(0);
+          if (n > 1) load_v(1);
+        }
+        __syncwarp();
+        // PROJ holds, in turn, PROJ_K(0), PROJ_Q(0), PROJ_K(1), PROJ_Q(1), ...; each fill
+        // waits until the previous one was read.
+        if (wait(sp_KT, 0)) proj(d_xk, sp_PROJK_FULL);
+        if (wait(sp_PROJK_READ, 0) && wait(sp_QT, 0)) proj(d_xq, sp_PROJQ_FULL);
+        if (n > 1 && wait(sp_PROJQ_READ, 0) && wait(sp_KT, 1)) proj(d_xk, sp_PROJK_FULL);
       }
-      // ---- state update, one bucket half per accumulator
-      if (!wait(sp_VT0 + (c & 1), (c >> 1) & 1)) break;
-      SW_TRACE(c, 4);
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t d_up0 = sdesc(pk_base + b0 * 32768, 16384, 1024, kSwizzle128B);
-        const uint64_t d_up1 = sdesc(pk_base + b1 * 32768, 16384, 1024, kSwizzle128B);
+      for (int c = 0; c < n && ok; ++c) {
+        const int i0 = 2 * c, i1 = 2 * c + 1;
+        const int b0 = i0 % 3, b1 = i1 % 3;
+        const uint32_t m0 = (uint32_t)(i0 / 3), m1 = (uint32_t)(i1 / 3);
+        const uint64_t d_vone = (c & 1) ? d_vone1 : d_vone0;
+        // ---- q projections of chunk c+1
+        if (c + 1 < n) {
+          if (!wait(sp_PROJK_READ, (c + 1) & 1)) break;
+          SW_TRACE(c, 7);
+          if (!wait(sp_QT, (c + 1) & 1)) break;
+          SW_TRACE(c, 8);
+          proj(d_xq, sp_PROJQ_FULL);
+        }
+        // ---- state update, one bucket half per accumulator
+        if (!wait(sp_PHK0 + b0, m0 & 1) || !wait(sp_PHK0 + b1, m1 & 1) ||
+            !wait(sp_VT0 + (c & 1), (c >> 1) & 1))
+          break;
+        if (c > 0 && !wait(sp_SREAD0, (c - 1) & 1)) break;
+        // the state update queues behind QK(c) and RO(c), which lie on the critical chains
+        if (!wait(sp_RO_ISSUED, c & 1)) break;
+        SW_TRACE(c, 4);
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t d_up0 = sdesc(pk_base + b0 * 32768, 16384, 1024, kSwizzle128B);
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ss(tmem + SPTm::S0, d_up0 + 128 * s, d_vone + vstep * s, id_up, 1);
-        umma_commit(bar + sp_UPD0);
-        umma_commit(bar + sp_KFREE0 + b0);
+          for (int s = 0; s < 8; ++s)
+            umma_ss(tmem + SPTm::S0, d_up0 + 128 * s, d_vone + vstep * s, id_up, 1);
+          umma_commit(bar + sp_UPD0);
+          umma_commit(bar + sp_KFREE0 + b0);
+        }
+        __syncwarp();
+        if (c > 0 && !wait(sp_SREAD1, (c - 1) & 1)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t d_up1 = sdesc(pk_base + b1 * 32768, 16384, 1024, kSwizzle128B);
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ss(tmem + SPTm::S1, d_up1 + 128 * s, d_vone + vstep * s, id_up, 1);
-        umma_commit(bar + sp_UPD1);
-        umma_commit(bar + sp_KFREE0 + b1);
+          for (int s = 0; s < 8; ++s)
+            umma_ss(tmem + SPTm::S1, d_up1 + 128 * s, d_vone + vstep * s, id_up, 1);
+          umma_commit(bar + sp_UPD1);
+          umma_commit(bar + sp_KFREE0 + b1);
+        }
+        __syncwarp();
+        // ---- k projections of chunk c+2
+        if (c + 2 < n) {
+          if (!wait(sp_PROJQ_READ, (c + 1) & 1) || !wait(sp_KT, c & 1)) break;
+          proj(d_xk, sp_PROJK_FULL);
+        }
+        SW_TRACE(c, 6);
       }
-      __syncwarp();
-      // ---- masked in-chunk weights times [v | 1]
-      if (!wait(sp_CONV, par)) break;
-      SW_TRACE(c, 5);
-      tc_fence_after();
-      if (elect_one()) {
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_ts(tmem + SPTm::num, tmem + SPTm::qk + s * 8, d_vone + vstep * s, id_ro, 1);
-        umma_commit(bar + sp_AV_DONE);
-      }
-      __syncwarp();
-      // ---- k projections of chunk c+2
-      if (c + 2 < n) {
-        if (!wait(sp_PROJQ_READ, (c + 1) & 1) || !wait(sp_KT, c & 1)) break;
-        proj(d_xk, sp_PROJK_FULL);
-      }
-      SW_TRACE(c, 6);
     }
   } else if (warp < 4) {
     // ================================================================ p(q) of chunk x
@@ -429,6 +477,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(bar + sp_PHQ0 + (g >> 2));
           if (t == 0) SW_TRACE(x, 12 + (g >> 2));
+          if (t == 96 && g == 7) SW_TRACE(x, 19);
         }
       }
     }
@@ -465,7 +514,9 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         const int i = 2 * x + half;
         const int b = i % 3;
         const int m = i / 3;
-        if (m >= 1 && !wait(sp_KFREE0 + b, (uint32_t)(m - 1) & 1)) break;
+        if (m >= 1 && (!wait(sp_KFREE0 + b, (uint32_t)(m - 1) & 1) ||
+                       !wait(sp_KFREEA0 + b, (uint32_t)(m - 1) & 1)))
+          break;
         if (t == 0) SW_TRACE(x, 21 + 2 * half);
         const uint32_t base = pk_base + b * 32768;
 #pragma unroll 1
@@ -483,6 +534,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar + sp_PHK0 + b);
         if (t == 0) SW_TRACE(x, 22 + 2 * half);
+        if (t == 96 && half == 1) SW_TRACE(x, 28);
       }
       if (!ok) break;
     }
@@ -495,6 +547,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       const uint32_t par = x & 1;
       if (!wait(sp_QK_FULL, par)) break;
       if (t == 0) SW_TRACE(x, 30);
+      if (t == 96) SW_TRACE(x, 14);
       tc_fence_after();
       // key block b (keys 32b..32b+31): blocks above this warp's rows are all zero
 #pragma unroll 1
@@ -505,6 +558,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           tmem_ld16(tmem + lane_off + SPTm::qk + 32 * b, f);
           tmem_ld16(tmem + lane_off + SPTm::qk + 32 * b + 16, f + 16);
           tmem_ld_wait();
+          if (t == 96 && b == 0) SW_TRACE(x, 15);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int j0 = 32 * b + 2 * e;
@@ -523,18 +577,37 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar + sp_CONV);
       if (t == 0) SW_TRACE(x, 31);
+      if (t == 96) SW_TRACE(x, 16);
+      // State halves: read into registers as soon as UPD(x) has written them (then UPD(x+1)
+      // may accumulate again), write the bf16 copy once RO(x) has read the previous one.
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {
         if (!wait(sp_UPD0 + hf, par)) break;
         tc_fence_after();
-        restage_row(tmem + lane_off + (hf ? SPTm::S1 : SPTm::S0), sb + SPSmem::sbf, 128 * hf + t);
+        uint32_t pk[40];
+        restage_load(tmem + lane_off + (hf ? SPTm::S1 : SPTm::S0), pk);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + sp_SREAD0 + hf);
+        if (t == 96 && hf == 0) SW_TRACE(x, 17);
+        if (t == 0 && hf == 0) SW_TRACE(x, 29);
+        if (hf == 0 && !wait(sp_PQ_FREE, par)) break;   // RO(x) read the state of chunk x-1
+        restage_store(sb + SPSmem::sbf, 128 * hf + t, pk);
         if (t == 0) SW_TRACE(x, 32 + hf);
+        if (t == 96) SW_TRACE(x, hf ? 34 : 18);
       }
       if (!ok) break;
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar + sp_SBF);
+      // v(x) was read by UPD(x) (waited above) and AV(x); v(x+2) takes its stage.  AV(x+1)
+      // needs this warp group's CONV(x+1), so AV_DONE cannot run a phase ahead here.
+      if (warp == 8 && x + 2 < n) {
+        if (!wait(sp_AV_DONE, par)) break;
+        if (elect_one()) load_v(x + 2);
+        __syncwarp();
+      }
     }
   } else {
     // ================================================================ output rows
@@ -548,8 +621,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       const int t0 = (int)(s0 + (int64_t)x * kC);
       if (!wait(sp_AV_DONE, x & 1)) break;
       if (t == 0) SW_TRACE(x, 35);
-      if (warp == 12 && x + 2 < n && elect_one()) load_v(x + 2);   // AV(x) read v(x) last
-      __syncwarp();
       tc_fence_after();
       uint32_t acc[72];
 #pragma unroll
@@ -585,6 +656,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  SW_TRACE_CTA(true);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
