@@ -263,25 +263,35 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (!ok && lane == 0) s_abort = 1;
       return ok;
     };
-    for (int i = 0; i < nchunks && ok; ++i) {
+    // x and feature tiles of sweep step i (one elected lane)
+    auto load_tiles = [&](int i) {
       const int c = REV ? nchunks - 1 - i : i;
       const int t0 = (int)(s0 + (int64_t)c * kC);
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar + kbTMA, (HAS_A ? 32768u : 0u) + (HAS_B ? 32768u : 0u));
-        if (HAS_A) {
-          tma_load_3d(sm + BwSmem::xa, &txa, 0, t0, h, bar + kbTMA);
+      mbar_arrive_expect_tx(bar + kbTMA, (HAS_A ? 32768u : 0u) + (HAS_B ? 32768u : 0u));
+      if (HAS_A) {
+        tma_load_3d(sm + BwSmem::xa, &txa, 0, t0, h, bar + kbTMA);
 #pragma unroll
-          for (int a = 0; a < 4; ++a)
-            tma_load_3d(sm + BwSmem::fa + a * 4096, &tfa, a * 16, t0, h, bar + kbTMA);
-        }
-        if (HAS_B) {
-          tma_load_3d(sm + BwSmem::xb, &txb, 0, t0, h, bar + kbTMA);
-#pragma unroll
-          for (int a = 0; a < 4; ++a)
-            tma_load_3d(sm + BwSmem::fb + a * 4096, &tfb, a * 16, t0, h, bar + kbTMA);
-        }
+        for (int a = 0; a < 4; ++a)
+          tma_load_3d(sm + BwSmem::fa + a * 4096, &tfa, a * 16, t0, h, bar + kbTMA);
       }
-      __syncwarp();
+      if (HAS_B) {
+        tma_load_3d(sm + BwSmem::xb, &txb, 0, t0, h, bar + kbTMA);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          tma_load_3d(sm + BwSmem::fb + a * 4096, &tfb, a * 16, t0, h, bar + kbTMA);
+      }
+    };
+    if (nchunks > 0 && elect_one()) load_tiles(0);
+    __syncwarp();
+    for (int i = 0; i < nchunks && ok; ++i) {
+      // With a state update, the tiles of step i+1 are loaded as soon as UPD(i) has
+      // completed (below), overlapping the copy and the projections with the CUDA-core
+      // warps' bf16 copy of the state.  Without one, once the step's work is done.
+      if (!HAS_B && i > 0) {
+        if (!wait(kbFREE, (i - 1) & 1)) break;
+        if (elect_one()) load_tiles(i);
+        __syncwarp();
+      }
       if (!wait(kbTMA, i & 1)) break;
       tc_fence_after();
       if (elect_one()) {
@@ -364,8 +374,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           umma_commit(bar + kbUP);
         }
         __syncwarp();
+        // every tile, p(b) and the projections of step i have been read once UPD(i) is
+        // done; the CUDA-core warps rewrite p(b) only after UPD(i) too, and arrive on PHI
+        // of step i+1 only after their copy of the state has been taken
+        if (!wait(kbUP, i & 1)) break;
+        if (i + 1 < nchunks && elect_one()) load_tiles(i + 1);
+        __syncwarp();
       }
-      if (!wait(kbFREE, i & 1)) break;
     }
   } else if (warp < 4) {
     // ================================================================ CUDA-core warps
@@ -512,7 +527,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
       tc_fence_before();
       named_bar(1, kAlu);
-      if (t == 0) mbar_arrive(bar + kbFREE);
+      if (!HAS_B && t == 0) mbar_arrive(bar + kbFREE);
     }
     if (MODE == kBuild && !s_abort) {
       float* out = seg_out + (((size_t)h * prm.n_rg + rg) * prm.G + g) * (size_t)256 * kNV;
