@@ -1033,7 +1033,7 @@ int64_t race_launch_count(void) { return launches::g_count.load(); }
 int race_sweep_trace_read(unsigned long long* dst) {
   cudaDeviceSynchronize();
   cudaMemcpyFromSymbol(dst, tc::g_sweep_trace, sizeof(tc::g_sweep_trace));
-  return tc::kTraceChunks * tc::kTraceEvents;
+  return 2 * tc::kTraceChunks * tc::kTraceEvents;
 }
 #endif
 

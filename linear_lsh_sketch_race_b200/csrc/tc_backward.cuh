@@ -58,7 +58,7 @@ struct BwTm {
 };
 
 enum BwBar : int {
-  kbTMA = 0, kbPROJ, kbPHI, kbDW, kbINTRA, kbDP, kbDPFREE, kbUP, kbFREE, kbCOUNT
+  kbTMAX = 0, kbTMAF, kbPROJ, kbPHI, kbDW, kbINTRA, kbDP, kbDPFREE, kbUP, kbFREE, kbCOUNT
 };
 
 // Extra feature columns of token row t in atom 4 of a 32B-swizzled feature tile.  The
@@ -67,12 +67,13 @@ enum BwBar : int {
 // keeps -(g . o)/den' to about 16 bits: it nearly cancels g . v / den' in dw_ij.  Zero
 // for tokens past the end.  The two 16-byte halves of a 32-byte row are swapped on rows
 // 4-7 of each 8-row group.
-__device__ __forceinline__ void store_extra_cols(uint32_t tile, int t, const float* e,
-                                                 size_t idx, bool valid) {
+// x: the extra value of the token on the g'' side (loaded ahead by the caller); ones:
+// the [v | 1] side.
+__device__ __forceinline__ void store_extra_cols(uint32_t tile, int t, float x, bool ones,
+                                                 bool valid) {
   float c0 = 0.f, c1 = 0.f;
   if (valid) {
-    if (e) {
-      const float x = e[idx];
+    if (!ones) {
       c0 = __bfloat162float(__float2bfloat16_rn(x));
       c1 = x - c0;
     } else {
@@ -87,13 +88,24 @@ __device__ __forceinline__ void store_extra_cols(uint32_t tile, int t, const flo
 
 // State row r as bf16 hi and bf16 lo = row - hi (X S^T adds both: the products with
 // g'' cancel to a small fraction of the state's size, so one bf16 rounding is too coarse).
+// Each pair is rounded once (one packed conversion); hi is widened back exactly by bit
+// moves, and lo = v - hi is exact in float32 before its own rounding.
 __device__ __forceinline__ void store_state_row_split(uint32_t hi_base, uint32_t lo_base, int r,
                                                       const float* v) {
-  float lo[kNV];
+  const uint32_t hb = hi_base + (r >> 3) * 1280 + (r & 7) * 16;
+  const uint32_t lb = lo_base + (r >> 3) * 1280 + (r & 7) * 16;
 #pragma unroll
-  for (int c = 0; c < kNV; ++c) lo[c] = v[c] - __bfloat162float(__float2bfloat16_rn(v[c]));
-  store_state_row_bf16(hi_base, r, v);
-  store_state_row_bf16(lo_base, r, lo);
+  for (int nc = 0; nc < 10; ++nc) {
+    uint32_t hp[4], lp[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = v[nc * 8 + 2 * e], b = v[nc * 8 + 2 * e + 1];
+      hp[e] = pack_bf16(a, b);
+      lp[e] = pack_bf16(a - __uint_as_float(hp[e] << 16), b - __uint_as_float(hp[e] & 0xffff0000u));
+    }
+    st_shared_v4(hb + nc * 128, hp[0], hp[1], hp[2], hp[3]);
+    st_shared_v4(lb + nc * 128, lp[0], lp[1], lp[2], lp[3]);
+  }
 }
 
 // Hash-backward partial sums of one token over the 128 sketch rows of half HALF.
@@ -263,36 +275,26 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (!ok && lane == 0) s_abort = 1;
       return ok;
     };
-    // x and feature tiles of sweep step i (one elected lane)
-    auto load_tiles = [&](int i) {
-      const int c = REV ? nchunks - 1 - i : i;
-      const int t0 = (int)(s0 + (int64_t)c * kC);
-      mbar_arrive_expect_tx(bar + kbTMA, (HAS_A ? 32768u : 0u) + (HAS_B ? 32768u : 0u));
-      if (HAS_A) {
-        tma_load_3d(sm + BwSmem::xa, &txa, 0, t0, h, bar + kbTMA);
+    // x tiles of sweep step i (read by PROJ(i) and by the CUDA-core warps' 1/|x| before
+    // PHI(i)) and feature tiles (read by the MMAs of step i up to UPD(i)); one elected lane
+    auto step_t0 = [&](int i) { return (int)(s0 + (int64_t)(REV ? nchunks - 1 - i : i) * kC); };
+    auto load_x = [&](int i) {
+      const int t0 = step_t0(i);
+      mbar_arrive_expect_tx(bar + kbTMAX, (HAS_A ? 16384u : 0u) + (HAS_B ? 16384u : 0u));
+      if (HAS_A) tma_load_3d(sm + BwSmem::xa, &txa, 0, t0, h, bar + kbTMAX);
+      if (HAS_B) tma_load_3d(sm + BwSmem::xb, &txb, 0, t0, h, bar + kbTMAX);
+    };
+    auto load_f = [&](int i) {
+      const int t0 = step_t0(i);
+      mbar_arrive_expect_tx(bar + kbTMAF, (HAS_A ? 16384u : 0u) + (HAS_B ? 16384u : 0u));
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-          tma_load_3d(sm + BwSmem::fa + a * 4096, &tfa, a * 16, t0, h, bar + kbTMA);
-      }
-      if (HAS_B) {
-        tma_load_3d(sm + BwSmem::xb, &txb, 0, t0, h, bar + kbTMA);
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-          tma_load_3d(sm + BwSmem::fb + a * 4096, &tfb, a * 16, t0, h, bar + kbTMA);
+      for (int a = 0; a < 4; ++a) {
+        if (HAS_A) tma_load_3d(sm + BwSmem::fa + a * 4096, &tfa, a * 16, t0, h, bar + kbTMAF);
+        if (HAS_B) tma_load_3d(sm + BwSmem::fb + a * 4096, &tfb, a * 16, t0, h, bar + kbTMAF);
       }
     };
-    if (nchunks > 0 && elect_one()) load_tiles(0);
-    __syncwarp();
-    for (int i = 0; i < nchunks && ok; ++i) {
-      // With a state update, the tiles of step i+1 are loaded as soon as UPD(i) has
-      // completed (below), overlapping the copy and the projections with the CUDA-core
-      // warps' bf16 copy of the state.  Without one, once the step's work is done.
-      if (!HAS_B && i > 0) {
-        if (!wait(kbFREE, (i - 1) & 1)) break;
-        if (elect_one()) load_tiles(i);
-        __syncwarp();
-      }
-      if (!wait(kbTMA, i & 1)) break;
+    // projections of the step whose x tiles are in shared memory
+    auto proj = [&]() {
       tc_fence_after();
       if (elect_one()) {
 #pragma unroll
@@ -313,7 +315,27 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         umma_commit(bar + kbPROJ);
       }
       __syncwarp();
+    };
+    if (nchunks > 0) {
+      if (elect_one()) {
+        load_x(0);
+        load_f(0);
+      }
+      __syncwarp();
+      if (wait(kbTMAX, 0)) proj();
+    }
+    // Step i: once the CUDA-core warps have read the projections and x tiles of step i
+    // (PHI), the x tiles of step i+1 are loaded; PROJ(i+1) is queued right behind the
+    // state update of step i, so it is done before the warps finish their copy of the
+    // state; the feature tiles of step i+1 follow the last MMA that reads step i's.
+    for (int i = 0; i < nchunks && ok; ++i) {
+      BW_TRACE(i, 0);
       if (!wait(kbPHI, i & 1)) break;
+      BW_TRACE(i, 2);
+      if (i + 1 < nchunks && elect_one()) load_x(i + 1);
+      __syncwarp();
+      if (!wait(kbTMAF, i & 1)) break;
+      BW_TRACE(i, 1);
       tc_fence_after();
       if (CAUSAL) {
         // X Y^T: rows of side a x tokens of side b, K = 80 feature columns
@@ -326,6 +348,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
         __syncwarp();
         if (!wait(kbINTRA, i & 1)) break;
+        BW_TRACE(i, 3);
         tc_fence_after();
       }
       if (HAS_A) {
@@ -357,6 +380,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           // this chunk's second half
           if (half == 0) {
             if (!wait(kbDPFREE, 0)) break;
+            BW_TRACE(i, 4);
             tc_fence_after();
           }
         }
@@ -374,25 +398,40 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           umma_commit(bar + kbUP);
         }
         __syncwarp();
-        // every tile, p(b) and the projections of step i have been read once UPD(i) is
-        // done; the CUDA-core warps rewrite p(b) only after UPD(i) too, and arrive on PHI
-        // of step i+1 only after their copy of the state has been taken
-        if (!wait(kbUP, i & 1)) break;
-        if (i + 1 < nchunks && elect_one()) load_tiles(i + 1);
-        __syncwarp();
       }
+      if (i + 1 < nchunks) {
+        if (!wait(kbTMAX, (i + 1) & 1)) break;
+        proj();
+      }
+      BW_TRACE(i, 5);
+      // the feature tiles of step i are free once UPD(i) (or, without a state update,
+      // the whole step) is done
+      if (HAS_B ? !wait(kbUP, i & 1) : !wait(kbFREE, i & 1)) break;
+      BW_TRACE(i, 6);
+      if (i + 1 < nchunks && elect_one()) load_f(i + 1);
+      __syncwarp();
     }
   } else if (warp < 4) {
     // ================================================================ CUDA-core warps
     const int t = threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int LP = prm.L * P;
+    // the g'' extra value of this thread's token, one step ahead (a global load)
+    const float* ex_src = HAS_A && ea ? ea : (HAS_B ? eb : nullptr);
+    auto load_ex = [&](int i) {
+      const int64_t row = s0 + (int64_t)(REV ? nchunks - 1 - i : i) * kC + t;
+      return (ex_src && row < s1) ? ex_src[(size_t)h * prm.N + row] : 0.f;
+    };
+    float ex_next = nchunks > 0 ? load_ex(0) : 0.f;
     for (int i = 0; i < nchunks; ++i) {
       if (s_abort) break;
       const int c = REV ? nchunks - 1 - i : i;
       const int64_t t0 = s0 + (int64_t)c * kC;
       const bool valid = (t0 + t) < s1;
+      const float ex = ex_next;
+      if (i + 1 < nchunks) ex_next = load_ex(i + 1);
       if (!mbar_wait(bar + kbPROJ, i & 1)) { s_abort = 1; break; }
+      if (t == 0) BW_TRACE(i, 10);
       tc_fence_after();
       float ua[NP], ub[NP];
       uint32_t r[16];
@@ -406,7 +445,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           for (int e = 0; e < 16; ++e) ua[b * 16 + e] = __uint_as_float(r[e]);
         }
         inv_a = row_inv_norm(sm + BwSmem::xa, t);
-        store_extra_cols(sb + BwSmem::fa, t, ea, (size_t)h * prm.N + t0 + t, valid);
+        store_extra_cols(sb + BwSmem::fa, t, ex, ea == nullptr, valid);
       }
       if (HAS_B) {
 #pragma unroll
@@ -418,40 +457,45 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
         const float sc = row_inv_norm(sm + BwSmem::xb, t) * prm.two_over_tau;
         write_phi_rows_rolled<P, TABLES>(sb + BwSmem::phb, t, ub, sc, valid);
-        store_extra_cols(sb + BwSmem::fb, t, eb, (size_t)h * prm.N + t0 + t, valid);
+        store_extra_cols(sb + BwSmem::fb, t, ex, eb == nullptr, valid);
       }
       fence_proxy_async();
       tc_fence_before();
       named_bar(1, kAlu);
       if (t == 0) mbar_arrive(bar + kbPHI);
+      if (t == 0) BW_TRACE(i, 11);
 
       if (CAUSAL) {
         // mask X Y^T (b tokens j <= t, or j >= t in the reverse sweep), round to bf16
         if (!mbar_wait(bar + kbDW, i & 1)) { s_abort = 1; break; }
+        if (t == 0) BW_TRACE(i, 12);
         tc_fence_after();
-        // key block kb (32 keys): loaded, masked and rounded before the next block's
-        // load; the bf16 pairs of block kb land in columns intra + 16 kb, which hold fp32
-        // keys already loaded (the first 64 fp32 columns)
+        // key blocks in pairs: blocks 0-1 (fp32 columns 0-63) are loaded, masked and
+        // rounded, and their bf16 pairs land in columns 0-31, which held keys already
+        // loaded; then blocks 2-3 (columns 64-127), whose pairs land in columns 32-63
 #pragma unroll 1
-        for (int kb = 0; kb < 4; ++kb) {
-          uint32_t x[32], o[16];
-          tmem_ld16(tmem + lane_off + BwTm::dw + kb * 32, x);
-          tmem_ld16(tmem + lane_off + BwTm::dw + kb * 32 + 16, x + 16);
+        for (int kp = 0; kp < 2; ++kp) {
+          uint32_t x[64], o[32];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tmem_ld16(tmem + lane_off + BwTm::dw + kp * 64 + q * 16, x + q * 16);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int j0 = kb * 32 + 2 * e;
+          for (int e = 0; e < 32; ++e) {
+            const int j0 = kp * 64 + 2 * e;
             const bool k0 = REV ? (j0 >= t) : (j0 <= t);
             const bool k1 = REV ? (j0 + 1 >= t) : (j0 + 1 <= t);
             o[e] = pack_bf16(k0 ? __uint_as_float(x[2 * e]) : 0.f,
                              k1 ? __uint_as_float(x[2 * e + 1]) : 0.f);
           }
-          tmem_st16(tmem + lane_off + BwTm::intra + kb * 16, o);
+          tmem_st16(tmem + lane_off + BwTm::intra + kp * 32, o);
+          tmem_st16(tmem + lane_off + BwTm::intra + kp * 32 + 16, o + 16);
         }
         tmem_st_wait();
         tc_fence_before();
         named_bar(1, kAlu);
         if (t == 0) mbar_arrive(bar + kbINTRA);
+        if (t == 0) BW_TRACE(i, 13);
       }
 
       if (HAS_A) {
@@ -484,6 +528,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!mbar_wait(bar + kbDP, half)) { s_abort = 1; break; }
+          if (t == 0) BW_TRACE(i, 14 + 2 * half);
           tc_fence_after();
           float dp[128];
 #pragma unroll
@@ -498,6 +543,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           tc_fence_before();
           named_bar(1, kAlu);
           if (t == 0) mbar_arrive(bar + kbDPFREE);
+          if (t == 0) BW_TRACE(i, 15 + 2 * half);
           if (half == 0) hash_bwd_half<P, 0>(dp, lo, hi, Ts, As);
           else hash_bwd_half<P, 1>(dp, lo, hi, Ts, As);
         }
@@ -514,6 +560,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 
       if (HAS_B) {
         if (!mbar_wait(bar + kbUP, i & 1)) { s_abort = 1; break; }
+        if (t == 0) BW_TRACE(i, 19);
         tc_fence_after();
         if (CAUSAL) {
 #pragma unroll 1
@@ -528,6 +575,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc_fence_before();
       named_bar(1, kAlu);
       if (!HAS_B && t == 0) mbar_arrive(bar + kbFREE);
+      if (t == 0) BW_TRACE(i, 20);
     }
     if (MODE == kBuild && !s_abort) {
       float* out = seg_out + (((size_t)h * prm.n_rg + rg) * prm.G + g) * (size_t)256 * kNV;

@@ -138,13 +138,15 @@ __device__ __forceinline__ void write_phi_rows(uint32_t tile, int t, int rows, i
 }
 
 // 1/max(|x|, eps) of token row t of a 128-byte-swizzled 128 x 64 bf16 tile (the
-// chunk order inside a row does not matter for a sum of squares).
+// chunk order inside a row does not matter for a sum of squares).  Thread t starts at
+// chunk t % 8, so eight consecutive rows (128 bytes apart) read eight different banks
+// groups in each step.
 __device__ __forceinline__ float row_inv_norm(const uint8_t* tile, int t) {
   const uint4* row = reinterpret_cast<const uint4*>(tile + t * 128);
   float s = 0.f;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    uint4 w = row[c];
+    uint4 w = row[c ^ (t & 7)];
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {

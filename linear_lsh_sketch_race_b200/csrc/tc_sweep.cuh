@@ -28,7 +28,8 @@ constexpr int kSwThreads = 288;
 // stamps per chunk and event, read back through race_sweep_trace_read().
 #ifdef RACE_SWEEP_TRACE
 constexpr int kTraceChunks = 512, kTraceEvents = 40;
-__device__ unsigned long long g_sweep_trace[kTraceChunks * kTraceEvents];
+// rows 0-511: forward sweep; rows 512-1023: backward sweep steps
+__device__ unsigned long long g_sweep_trace[2 * kTraceChunks * kTraceEvents];
 #define SW_TRACE(c, ev)                                                                 \
   do {                                                                                  \
     if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (c) < kTraceChunks)    \
@@ -49,12 +50,20 @@ __device__ __forceinline__ void sw_trace_cta(bool end) {
   r[25] = sm;
 }
 #define SW_TRACE_CTA(end) sw_trace_cta(end)
+#define BW_TRACE(c, ev)                                                                 \
+  do {                                                                                  \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (c) < kTraceChunks)    \
+      g_sweep_trace[(kTraceChunks + (c)) * kTraceEvents + (ev)] = clock64();             \
+  } while (0)
 #else
 #define SW_TRACE(c, ev) \
   do {                  \
   } while (0)
 #define SW_TRACE_CTA(end) \
   do {                    \
+  } while (0)
+#define BW_TRACE(c, ev) \
+  do {                  \
   } while (0)
 #endif
 
