@@ -58,7 +58,7 @@ struct BwTm {
 };
 
 enum BwBar : int {
-  kbTMAX = 0, kbTMAF, kbPROJ, kbPHI, kbDW, kbINTRA, kbDP, kbDPFREE, kbUP, kbFREE, kbCOUNT
+  kbTMAX = 0, kbTMAF, kbPROJ, kbPHI, kbDW, kbINTRA, kbDP, kbDPFREE, kbUP, kbCOUNT
 };
 
 // Extra feature columns of token row t in atom 4 of a 32B-swizzled feature tile.  The
@@ -324,10 +324,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       __syncwarp();
       if (wait(kbTMAX, 0)) proj();
     }
-    // Step i: once the CUDA-core warps have read the projections and x tiles of step i
-    // (PHI), the x tiles of step i+1 are loaded; PROJ(i+1) is queued right behind the
-    // state update of step i, so it is done before the warps finish their copy of the
-    // state; the feature tiles of step i+1 follow the last MMA that reads step i's.
+    // Step i in tensor-core order: X Y^T, UPD (while the CUDA-core warps mask X Y^T),
+    // dP half 0, dP half 1, PROJ(i+1).  The x tiles of step i+1 are loaded once the
+    // warps have read the projections and x tiles of step i (PHI); PROJ(i+1) follows
+    // every MMA of step i, and its completion frees the feature tiles for step i+1.
     for (int i = 0; i < nchunks && ok; ++i) {
       BW_TRACE(i, 0);
       if (!wait(kbPHI, i & 1)) break;
@@ -347,6 +347,24 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           umma_commit(bar + kbDW);
         }
         __syncwarp();
+      }
+      if (HAS_B) {
+        // S += p(b)^T Y, both halves of the sketch rows (K = 128 tokens); it runs while
+        // the CUDA-core warps mask X Y^T.  dP(i) reads the bf16 copy of the state before
+        // step i, which the warps rewrite only after dP(i) (and this update) are done.
+        tc_fence_after();
+        if (elect_one()) {
+          for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+              umma_ss(tmem + (half ? BwTm::S1 : BwTm::S0),
+                      sdesc(sb + BwSmem::phb + half * 2048 + s * 8192, 4096, 128, kSwizzleNone),
+                      sdesc(sb + BwSmem::fb + s * 512, 4096, 256, kSwizzle32B), id_up, 1);
+          umma_commit(bar + kbUP);
+        }
+        __syncwarp();
+      }
+      if (CAUSAL) {
         if (!wait(kbINTRA, i & 1)) break;
         BW_TRACE(i, 3);
         tc_fence_after();
@@ -376,8 +394,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             umma_commit(bar + kbDP);
           }
           __syncwarp();
-          // the next chunk's first half waits for FREE, which follows the release of
-          // this chunk's second half
+          // the second half overwrites dP once the warps have read the first; the next
+          // step's first half comes after its PHI, i.e. after the warps read this one's
+          // second half
           if (half == 0) {
             if (!wait(kbDPFREE, 0)) break;
             BW_TRACE(i, 4);
@@ -386,30 +405,17 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
         if (!ok) break;
       }
-      if (HAS_B) {
-        // S += p(b)^T Y, both halves of the sketch rows (K = 128 tokens)
-        if (elect_one()) {
-          for (int half = 0; half < 2; ++half)
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-              umma_ss(tmem + (half ? BwTm::S1 : BwTm::S0),
-                      sdesc(sb + BwSmem::phb + half * 2048 + s * 8192, 4096, 128, kSwizzleNone),
-                      sdesc(sb + BwSmem::fb + s * 512, 4096, 256, kSwizzle32B), id_up, 1);
-          umma_commit(bar + kbUP);
-        }
-        __syncwarp();
-      }
       if (i + 1 < nchunks) {
         if (!wait(kbTMAX, (i + 1) & 1)) break;
         proj();
+        BW_TRACE(i, 5);
+        // PROJ(i+1) follows every MMA of step i, so its completion frees the feature
+        // tiles of step i (the CUDA-core warps wait on the same barrier)
+        if (!wait(kbPROJ, (i + 1) & 1)) break;
+        BW_TRACE(i, 6);
+        if (elect_one()) load_f(i + 1);
+        __syncwarp();
       }
-      BW_TRACE(i, 5);
-      // the feature tiles of step i are free once UPD(i) (or, without a state update,
-      // the whole step) is done
-      if (HAS_B ? !wait(kbUP, i & 1) : !wait(kbFREE, i & 1)) break;
-      BW_TRACE(i, 6);
-      if (i + 1 < nchunks && elect_one()) load_f(i + 1);
-      __syncwarp();
     }
   } else if (warp < 4) {
     // ================================================================ CUDA-core warps
@@ -434,27 +440,26 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (t == 0) BW_TRACE(i, 10);
       tc_fence_after();
       float ua[NP], ub[NP];
-      uint32_t r[16];
       float inv_a = 0.f;
-      if (HAS_A) {
+      {   // both sides' projections: all loads in flight, one wait
+        uint32_t ra[NP], rb[NP];
 #pragma unroll
         for (int b = 0; b < NP / 16; ++b) {
-          tmem_ld16(tmem + lane_off + BwTm::pa + b * 16, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ua[b * 16 + e] = __uint_as_float(r[e]);
+          if (HAS_A) tmem_ld16(tmem + lane_off + BwTm::pa + b * 16, ra + b * 16);
+          if (HAS_B) tmem_ld16(tmem + lane_off + BwTm::pb + b * 16, rb + b * 16);
         }
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+          ua[e] = HAS_A ? __uint_as_float(ra[e]) : 0.f;
+          ub[e] = HAS_B ? __uint_as_float(rb[e]) : 0.f;
+        }
+      }
+      if (HAS_A) {
         inv_a = row_inv_norm(sm + BwSmem::xa, t);
         store_extra_cols(sb + BwSmem::fa, t, ex, ea == nullptr, valid);
       }
       if (HAS_B) {
-#pragma unroll
-        for (int b = 0; b < NP / 16; ++b) {
-          tmem_ld16(tmem + lane_off + BwTm::pb + b * 16, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ub[b * 16 + e] = __uint_as_float(r[e]);
-        }
         const float sc = row_inv_norm(sm + BwSmem::xb, t) * prm.two_over_tau;
         write_phi_rows_rolled<P, TABLES>(sb + BwSmem::phb, t, ub, sc, valid);
         store_extra_cols(sb + BwSmem::fb, t, ex, eb == nullptr, valid);
@@ -550,11 +555,20 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         if (s_abort) break;
         if (valid) {
           float* dst = du_out + ((size_t)h * prm.N + t0 + t) * LP + (size_t)l0 * P;
+          float d[TABLES * P];
 #pragma unroll
           for (int j = 0; j < TABLES; ++j)
 #pragma unroll
             for (int p = 0; p < P; ++p)
-              dst[j * P + p] = prm.two_over_tau * (As[j * P + p] - sp[j * P + p] * Ts[j]);
+              d[j * P + p] = prm.two_over_tau * (As[j * P + p] - sp[j * P + p] * Ts[j]);
+          if ((TABLES * P) % 4 == 0) {   // the row group's slice is then 16-byte aligned
+#pragma unroll
+            for (int e = 0; e < TABLES * P; e += 4)
+              *reinterpret_cast<float4*>(dst + e) = make_float4(d[e], d[e + 1], d[e + 2], d[e + 3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < TABLES * P; ++e) dst[e] = d[e];
+          }
         }
       }
 
@@ -574,7 +588,6 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
       tc_fence_before();
       named_bar(1, kAlu);
-      if (!HAS_B && t == 0) mbar_arrive(bar + kbFREE);
       if (t == 0) BW_TRACE(i, 20);
     }
     if (MODE == kBuild && !s_abort) {

@@ -143,7 +143,7 @@ __device__ __forceinline__ void write_phi_rows(uint32_t tile, int t, int rows, i
 // groups in each step.
 __device__ __forceinline__ float row_inv_norm(const uint8_t* tile, int t) {
   const uint4* row = reinterpret_cast<const uint4*>(tile + t * 128);
-  float s = 0.f;
+  float s[4] = {0.f, 0.f, 0.f, 0.f};   // four independent sums: short dependency chains
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     uint4 w = row[c ^ (t & 7)];
@@ -152,10 +152,10 @@ __device__ __forceinline__ float row_inv_norm(const uint8_t* tile, int t) {
     for (int e = 0; e < 4; ++e) {
       __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&ws[e]);
       float2 f = __bfloat1622float2(b2);
-      s = fmaf(f.x, f.x, fmaf(f.y, f.y, s));
+      s[e] = fmaf(f.x, f.x, fmaf(f.y, f.y, s[e]));
     }
   }
-  return 1.0f / fmaxf(sqrtf(s), kEpsNorm);
+  return 1.0f / fmaxf(sqrtf((s[0] + s[1]) + (s[2] + s[3])), kEpsNorm);
 }
 
 // bf16 copy of one 80-column state row into the readout B operand (MN-major, no
