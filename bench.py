@@ -78,12 +78,34 @@ def kernel_work(name: str, wl: I.Workload):
         "simt_bwd_q": 4 * LR * (d + 1) + 8 * d * L * P,
         "simt_bwd_kv": 6 * LR * (d + 1) + 8 * d * L * P,
         "tc_causal_sweep": 4 * LR * (d + 1) + 4 * d * L * P,
+        # q side: state of p(k)[v | 1] plus its readout by g'' (dP of p(q)); k side: the
+        # same with the roles exchanged; both also project q and k
+        "tc_bwd_q": 4 * LR * (d + 1) + 4 * d * L * P,
+        "tc_bwd_k": 4 * LR * (d + 1) + 4 * d * L * P,
         "tc_sketch_build": 2 * LR * (d + 1) + 2 * d * L * P,
         "tc_readout": 2 * LR * (d + 1) + 2 * d * L * P,
     }
     if name not in table:
         return None
     return table[name] * th
+
+
+# DRAM bytes (read + write) per token-head of a launch, from one ncu capture of a smaller
+# launch of the same kernel and configuration (8 heads, N = 131,072, L = 16, P = 8; full
+# set, `dram__bytes_read.sum + dram__bytes_write.sum`): 946 MB for the forward sweep and
+# 1,319 MB for the q side of the backward sweep (the k side is the same kernel with the
+# roles of the two sides exchanged).  The traffic grows in proportion to H x N.
+DRAM_BYTES_PER_TOKEN_HEAD = {
+    "tc_causal_sweep": 946.05e6 / (8 * 131072),
+    "tc_bwd_q": 1319.13e6 / (8 * 131072),
+    "tc_bwd_k": 1319.13e6 / (8 * 131072),
+}
+
+
+def kernel_traffic(name: str, wl: I.Workload):
+    if wl.L != 16 or wl.P != 8 or name not in DRAM_BYTES_PER_TOKEN_HEAD:
+        return None
+    return DRAM_BYTES_PER_TOKEN_HEAD[name] * wl.H * wl.N
 
 
 def rank_heads(rank: int, heads_per_rank: int):
@@ -297,20 +319,25 @@ def run_ours(args, wl: I.Workload):
     peaks, peak_src = load_peaks()
     f_fwd, f_bwd = flops_per_token_head(wl)
 
-    # dominant kernel of the step, against the sustained tensor peak
-    roof = None
-    cands = [(t[0], n) for n, t in ktimes.items() if kernel_work(n, wl) is not None]
-    if cands:
-        tot, name = max(cands)
+    # dominant kernel of the step (and the forward sweep), against the sustained tensor peak
+    def roofline_of(name):
         ms_launch = ktimes[name][0] / ktimes[name][1]
         work = kernel_work(name, wl)
         achieved = work / (ms_launch / 1000) / 1e12
         peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+        return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": kernel_traffic(name, wl),
                 "peak_source": f"{peak_src} bf16_tflops_sustained",
                 "ms_per_launch": ms_launch, "flops_per_launch": work,
-                "share_of_step": tot / sum(t[0] for t in ktimes.values())}
+                "share_of_step": ktimes[name][0] / sum(t[0] for t in ktimes.values())}
+
+    roof = roof_fwd = None
+    cands = [(t[0], n) for n, t in ktimes.items() if kernel_work(n, wl) is not None]
+    if cands:
+        roof = roofline_of(max(cands)[1])
+    if "tc_causal_sweep" in ktimes and roof and roof["kernel"] != "tc_causal_sweep":
+        roof_fwd = roofline_of("tc_causal_sweep")
 
     ideal_ms = max(wl.H * wl.N * (f_fwd + (f_bwd if backward else 0)) /
                    (peaks["bf16_tflops"] * 1e12),
@@ -332,6 +359,7 @@ def run_ours(args, wl: I.Workload):
         "method_roofline": {"ideal_ms_per_step": ideal_ms, "frac": ideal_ms / ms,
                             "peak_source": f"{peak_src} bf16_tflops (burst) / hbm_gbs"},
         "roofline": roof,
+        "roofline_fwd_sweep": roof_fwd,
         "kernel_ms_per_step": {n: t[0] / args.steps for n, t in ktimes.items()},
         "gpu_launches": launches,
         "clocks": clocks,
