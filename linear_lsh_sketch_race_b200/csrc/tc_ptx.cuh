@@ -221,6 +221,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// bf16 pair (h * lo2.x, h * lo2.y): one packed float multiply and one packed conversion,
+// the same roundings as two float multiplies and a conversion.
+__device__ __forceinline__ uint32_t mul_pack_bf16(uint64_t lo2, uint64_t hh) {
+  uint32_t out;
+  asm("{\n\t.reg .b64 pr;\n\t.reg .f32 a, b;\n\t"
+      "mul.rn.f32x2 pr, %1, %2;\n\t"
+      "mov.b64 {a, b}, pr;\n\t"
+      "cvt.rn.bf16x2.f32 %0, b, a;\n\t}"
+      : "=r"(out)
+      : "l"(lo2), "l"(hh));
+  return out;
+}
+__device__ __forceinline__ uint64_t bcast_f32x2(float h) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(h));
+  return r;
+}
+__device__ __forceinline__ uint64_t pair_f32x2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),

@@ -111,29 +111,6 @@ struct Corners {
   uint64_t lo2[4];   // float pairs (lo[2e], lo[2e+1]) in one 64-bit register
 };
 
-// bf16 pair (h * lo2.x, h * lo2.y): one packed float multiply and one packed conversion,
-// the same roundings as two float multiplies and a conversion.
-__device__ __forceinline__ uint32_t mul_pack_bf16(uint64_t lo2, uint64_t hh) {
-  uint32_t out;
-  asm("{\n\t.reg .b64 pr;\n\t.reg .f32 a, b;\n\t"
-      "mul.rn.f32x2 pr, %1, %2;\n\t"
-      "mov.b64 {a, b}, pr;\n\t"
-      "cvt.rn.bf16x2.f32 %0, b, a;\n\t}"
-      : "=r"(out)
-      : "l"(lo2), "l"(hh));
-  return out;
-}
-__device__ __forceinline__ uint64_t bcast_f32x2(float h) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(h));
-  return r;
-}
-__device__ __forceinline__ uint64_t pair_f32x2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-
 __device__ __forceinline__ void corners_of(const float* sp, const float* sm, float valid,
                                            Corners& k) {
 #pragma unroll
