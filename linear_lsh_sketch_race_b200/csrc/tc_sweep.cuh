@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       const int64_t t0 = s0 + (int64_t)c * kC;
       const float valid = (t0 + t) < s1 ? 1.f : 0.f;
       // ---- projections and norms
-      const int eb = 10 + 15 * grp;
+      [[maybe_unused]] const int eb = 10 + 15 * grp;   // trace events of this group
       if (t == 0) SW_TRACE(c, eb + 0);
       if (!wait(kB_PROJ, par)) break;
       if (t == 0) SW_TRACE(c, eb + 1);

@@ -319,7 +319,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           mbar_arrive(bar + sp_RO_ISSUED);
         }
         __syncwarp();
-        SW_TRACE(c, 9);
         // ---- masked in-chunk weights times [v | 1]
         if (!wait(sp_CONV, par) || !wait(sp_VT0 + (c & 1), (c >> 1) & 1)) break;
         SW_TRACE(c, 5);
@@ -362,10 +361,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         const uint64_t d_vone = (c & 1) ? d_vone1 : d_vone0;
         // ---- q projections of chunk c+1
         if (c + 1 < n) {
-          if (!wait(sp_PROJK_READ, (c + 1) & 1)) break;
-          SW_TRACE(c, 7);
-          if (!wait(sp_QT, (c + 1) & 1)) break;
-          SW_TRACE(c, 8);
+          if (!wait(sp_PROJK_READ, (c + 1) & 1) || !wait(sp_QT, (c + 1) & 1)) break;
           proj(d_xq, sp_PROJQ_FULL);
         }
         // ---- state update, one bucket half per accumulator
@@ -454,7 +450,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(bar + sp_PHQ0 + (g >> 2));
           if (t == 0) SW_TRACE(x, 12 + (g >> 2));
-          if (t == 96 && g == 7) SW_TRACE(x, 19);
         }
       }
     }
@@ -511,7 +506,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar + sp_PHK0 + b);
         if (t == 0) SW_TRACE(x, 22 + 2 * half);
-        if (t == 96 && half == 1) SW_TRACE(x, 28);
       }
       if (!ok) break;
     }
@@ -524,7 +518,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       const uint32_t par = x & 1;
       if (!wait(sp_QK_FULL, par)) break;
       if (t == 0) SW_TRACE(x, 30);
-      if (t == 96) SW_TRACE(x, 14);
       tc_fence_after();
       // key block b (keys 32b..32b+31): blocks above this warp's rows are all zero
 #pragma unroll 1
@@ -535,7 +528,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           tmem_ld16(tmem + lane_off + SPTm::qk + 32 * b, f);
           tmem_ld16(tmem + lane_off + SPTm::qk + 32 * b + 16, f + 16);
           tmem_ld_wait();
-          if (t == 96 && b == 0) SW_TRACE(x, 15);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int j0 = 32 * b + 2 * e;
@@ -554,7 +546,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar + sp_CONV);
       if (t == 0) SW_TRACE(x, 31);
-      if (t == 96) SW_TRACE(x, 16);
       // State halves: read into registers as soon as UPD(x) has written them (then UPD(x+1)
       // may accumulate again), write the bf16 copy once RO(x) has read the previous one.
 #pragma unroll 1
@@ -566,12 +557,9 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar + sp_SREAD0 + hf);
-        if (t == 96 && hf == 0) SW_TRACE(x, 17);
-        if (t == 0 && hf == 0) SW_TRACE(x, 29);
         if (hf == 0 && !wait(sp_PQ_FREE, par)) break;   // RO(x) read the state of chunk x-1
         restage_store(sb + SPSmem::sbf, 128 * hf + t, pk);
         if (t == 0) SW_TRACE(x, 32 + hf);
-        if (t == 96) SW_TRACE(x, hf ? 34 : 18);
       }
       if (!ok) break;
       fence_proxy_async();
