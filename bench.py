@@ -108,6 +108,32 @@ def kernel_traffic(name: str, wl: I.Workload):
     return DRAM_BYTES_PER_TOKEN_HEAD[name] * wl.H * wl.N
 
 
+def roofline_lines(ktimes, wl: I.Workload, peaks, peak_src: str):
+    """Roofline objects of the JSON line from the per-kernel CUDA-event totals
+    ktimes = {name: (total_ms, launches)}: the dominant kernel of the step (the largest
+    total among kernels with known algorithmic work) and, when that is not the forward
+    sweep, the forward sweep as well; both against the sustained tensor peak."""
+    def roofline_of(name):
+        ms_launch = ktimes[name][0] / ktimes[name][1]
+        work = kernel_work(name, wl)
+        achieved = work / (ms_launch / 1000) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": kernel_traffic(name, wl),
+                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "ms_per_launch": ms_launch, "flops_per_launch": work,
+                "share_of_step": ktimes[name][0] / sum(t[0] for t in ktimes.values())}
+
+    roof = roof_fwd = None
+    cands = [(t[0], n) for n, t in ktimes.items() if kernel_work(n, wl) is not None]
+    if cands:
+        roof = roofline_of(max(cands)[1])
+    if "tc_causal_sweep" in ktimes and roof and roof["kernel"] != "tc_causal_sweep":
+        roof_fwd = roofline_of("tc_causal_sweep")
+    return roof, roof_fwd
+
+
 def rank_heads(rank: int, heads_per_rank: int):
     """Global head indices of one rank: heads are independent (W is shared), so with weak
     scaling rank r owns heads r*H .. r*H + H - 1 of the global batch of heads."""
@@ -319,25 +345,7 @@ def run_ours(args, wl: I.Workload):
     peaks, peak_src = load_peaks()
     f_fwd, f_bwd = flops_per_token_head(wl)
 
-    # dominant kernel of the step (and the forward sweep), against the sustained tensor peak
-    def roofline_of(name):
-        ms_launch = ktimes[name][0] / ktimes[name][1]
-        work = kernel_work(name, wl)
-        achieved = work / (ms_launch / 1000) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": kernel_traffic(name, wl),
-                "peak_source": f"{peak_src} bf16_tflops_sustained",
-                "ms_per_launch": ms_launch, "flops_per_launch": work,
-                "share_of_step": ktimes[name][0] / sum(t[0] for t in ktimes.values())}
-
-    roof = roof_fwd = None
-    cands = [(t[0], n) for n, t in ktimes.items() if kernel_work(n, wl) is not None]
-    if cands:
-        roof = roofline_of(max(cands)[1])
-    if "tc_causal_sweep" in ktimes and roof and roof["kernel"] != "tc_causal_sweep":
-        roof_fwd = roofline_of("tc_causal_sweep")
+    roof, roof_fwd = roofline_lines(ktimes, wl, peaks, peak_src)
 
     ideal_ms = max(wl.H * wl.N * (f_fwd + (f_bwd if backward else 0)) /
                    (peaks["bf16_tflops"] * 1e12),
