@@ -422,7 +422,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int t = threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int LP = prm.L * P;
-    // the g'' extra value of this thread's token, one step ahead (a global load)
+    // the g'' extra value of this thread's token, one step ahead (a global load); at most
+    // one side is the g'' side (ea or eb non-null), the other is [v | 1]
     const float* ex_src = HAS_A && ea ? ea : (HAS_B ? eb : nullptr);
     auto load_ex = [&](int i) {
       const int64_t row = s0 + (int64_t)(REV ? nchunks - 1 - i : i) * kC + t;
