@@ -134,6 +134,15 @@ def roofline_lines(ktimes, wl: I.Workload, peaks, peak_src: str):
     return roof, roof_fwd
 
 
+def chunk_ran(wl: I.Workload, kernels: str) -> int:
+    """Tokens per chunk of the kernels that run: the tensor-core sweeps use 128-token chunks
+    (bf16, 6 <= P <= 8, L * 2^P a multiple of 128), the CUDA-core kernels 32-token tiles;
+    the workload's requested chunk is advisory."""
+    tensor = (wl.dtype == "bf16" and kernels != "simt" and 6 <= wl.P <= 8
+              and (wl.L << wl.P) % 128 == 0)
+    return 128 if tensor else 32
+
+
 def rank_heads(rank: int, heads_per_rank: int):
     """Global head indices of one rank: heads are independent (W is shared), so with weak
     scaling rank r owns heads r*H .. r*H + H - 1 of the global batch of heads."""
@@ -357,7 +366,8 @@ def run_ours(args, wl: I.Workload):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": wl.name, "H": wl.H, "N": wl.N, "d": wl.d, "L": wl.L,
-                   "P": wl.P, "tau": wl.tau, "causal": wl.causal, "chunk": wl.chunk,
+                   "P": wl.P, "tau": wl.tau, "causal": wl.causal,
+                   "chunk": chunk_ran(wl, args.kernels), "chunk_requested": wl.chunk,
                    "step": "fwd+bwd" if backward else "fwd", "kernels": args.kernels,
                    "l2": "inputs larger than L2 (q, k, v = %.1f GB per rank)" %
                          (3 * q.numel() * q.element_size() / 1e9),

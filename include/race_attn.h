@@ -70,7 +70,11 @@ typedef enum { RACE_BF16 = 0, RACE_FP32 = 1 } race_dtype_t;
 /* Which kernels a call may use.  AUTO picks the tensor-core (tcgen05) path for
  * bf16 inputs where it exists and the CUDA-core path otherwise.  SIMT forces the
  * CUDA-core kernels (always available; the only path for fp32).  TENSOR forces the
- * tensor-core kernels and fails with RACE_ERR_UNSUPPORTED where they do not apply. */
+ * tensor-core kernels and fails with RACE_ERR_UNSUPPORTED where they do not apply.
+ * The tensor-core kernels cover bf16 inputs with 6 <= P <= 8 and N < 2^31 - 128, and
+ *   forward:  L * 2^P a multiple of 128;
+ *   backward: L * 2^P a multiple of 256 and L * P <= 256.
+ * Every other shape runs on the CUDA-core kernels under AUTO. */
 typedef enum { RACE_IMPL_AUTO = 0, RACE_IMPL_SIMT = 1, RACE_IMPL_TENSOR = 2 } race_impl_t;
 
 /* Full argument set of the *_ex entry points. */
@@ -82,21 +86,25 @@ typedef struct {
   int P;                     /* hyperplanes per table; R = 2^P buckets                 */
   float tau;                 /* soft-hash temperature (the pages' beta is 1/tau)       */
   int causal;                /* 0: all keys; 1: keys j <= i                            */
-  race_dtype_t dtype;        /* element type of q, k, v, dout, dq, dk, dv              */
+  race_dtype_t dtype;        /* element type of q, k, v, dout                          */
   race_dtype_t out_dtype;    /* element type of out (forward writes, backward reads)   */
-  int chunk;                 /* tokens per chunk of the causal sweep; 0 = library      */
-                             /* choice; otherwise a multiple of 64 (tensor-core path)   */
-                             /* or of 32 (CUDA-core path)                               */
+  int chunk;                 /* advisory tokens per chunk: 0 or a positive multiple of  */
+                             /* 32 (others: RACE_ERR_INVALID_ARG).  The tensor-core     */
+                             /* kernels always run 128-token chunks and the CUDA-core   */
+                             /* kernels 32-token tiles; results do not depend on it     */
   void *workspace;           /* device scratch of >= workspace_bytes, or NULL: the      */
   size_t workspace_bytes;    /* library then allocates stream-ordered scratch itself    */
   float *den;                /* optional [H][N]: forward writes den_i =                 */
                              /* sum_j phi(q_i).phi(k_j); backward reads it (NULL: the   */
                              /* backward recomputes it)                                 */
   race_impl_t impl;          /* kernel family, see race_impl_t                          */
+  race_dtype_t grad_dtype;   /* element type of dq, dk, dv written by the backward      */
+                             /* (bf16 or float32, for either input dtype; float32 keeps */
+                             /* the gradients free of a final bf16 rounding)            */
 } race_args_t;
 
-/* Fill `a` with the defaults of the spec-form calls: bf16 in and out, chunk 0,
- * no workspace, no den, RACE_IMPL_AUTO. */
+/* Fill `a` with the defaults of the spec-form calls: bf16 in, out and gradients,
+ * chunk 0, no workspace, no den, RACE_IMPL_AUTO. */
 void race_args_init(race_args_t *a, int64_t N, int H, int d, int L, int P, float tau,
                     int causal);
 
@@ -147,9 +155,9 @@ race_status_t race_backward_ex(const void *q, const void *k, const void *v,
  * device).  No cudaMalloc, cudaMallocAsync or other allocating routine is called; the
  * call clears the parts of the array that must start at zero on `stream` itself.
  *
- * Set-up: the first call on each device looks up the array's device address (with
- * that device current) and may load the module there.  Make that first call before
- * any stream capture begins.
+ * Set-up: every call looks up the array's device address on the current device (so a
+ * device reset cannot leave a stale address behind); the first call on a device may
+ * load the module there.  Make that first call before any stream capture begins.
  *
  * Concurrency: all calls on one device share the array.  Calls that can overlap in
  * time (different streams, or different host threads without ordering) race on it and
@@ -184,6 +192,21 @@ race_status_t race_hash(const void *x, const float *W, void *phi, const race_arg
  * NULL) receives the raw flag bits.  Returns RACE_OK or RACE_ERR_DEVICE_STATUS (or
  * RACE_ERR_CUDA). */
 race_status_t race_device_status(race_stream_t stream, uint32_t *flags);
+
+/* ---------------------------------------------------------------------------------
+ * race_selftest_wait_timeout — exercises the failure path of the library's kernels
+ * without any fault: one kernel (a single warp; no TMA copy, no MMA) waits on an
+ * mbarrier phase that nothing completes, through the same bounded-wait routine the
+ * tensor-core kernels use, with a limit of `limit_cycles` SM clock cycles
+ * (1 <= limit_cycles <= 2e9, the kernels' own limit; about 1e6 is half a millisecond).
+ * The wait gives up, raises the timeout bit (1) of the device status flag and the
+ * kernel returns, so the context stays usable.  Synchronises `stream`; *timed_out
+ * (host, may be NULL) receives 1 when every lane gave up.  The flag stays raised for
+ * race_device_status to report (RACE_ERR_DEVICE_STATUS) and clear.
+ * Returns RACE_OK, RACE_ERR_INVALID_ARG or RACE_ERR_CUDA.
+ * ------------------------------------------------------------------------------ */
+race_status_t race_selftest_wait_timeout(int64_t limit_cycles, int *timed_out,
+                                         race_stream_t stream);
 
 /* Static description of a status code. */
 const char *race_status_string(race_status_t s);

@@ -1,9 +1,12 @@
 // C-ABI implementation of librace_attn.so: argument checks, planning, scratch
 // layout and kernel launches.  The whole library is one translation unit so that the
 // device status flag is a single __device__ symbol.
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -16,8 +19,36 @@
 #include "tc_sweep.cuh"
 #include "tc_sweep_pipe.cuh"
 #include "tc_backward.cuh"
+#include "tc_finalize.cuh"
 
 namespace race {
+
+// ------------------------------------------------------------------ NVTX (opt-in)
+// With RACE_NVTX=1 in the environment (read once), every entry point and every kernel
+// launch of the library is bracketed by an NVTX range named after it, for timeline
+// tools.  Off by default: no NVTX call is made.
+inline bool nvtx_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("RACE_NVTX");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
+
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) : on_(nvtx_enabled()) {
+    if (on_) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on_) nvtxRangePop();
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+
+ private:
+  bool on_;
+};
 
 // ------------------------------------------------------------------ launch accounting
 // Every kernel launch of the library goes through a LaunchScope: it counts launches
@@ -73,7 +104,7 @@ void drain() {
 
 class Scope {
  public:
-  Scope(const char* name, cudaStream_t s) : name_(name), s_(s) {
+  Scope(const char* name, cudaStream_t s) : name_(name), s_(s), range_(name) {
     g_count.fetch_add(1, std::memory_order_relaxed);
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_timing) {
@@ -92,6 +123,7 @@ class Scope {
  private:
   const char* name_;
   cudaStream_t s_;
+  NvtxRange range_;
   cudaEvent_t start_ = nullptr, stop_ = nullptr;
 };
 
@@ -120,7 +152,8 @@ race_status_t check_args(const race_args_t* a) {
     return RACE_ERR_INVALID_ARG;
   if (a->impl != RACE_IMPL_AUTO && a->impl != RACE_IMPL_SIMT && a->impl != RACE_IMPL_TENSOR)
     return RACE_ERR_INVALID_ARG;
-  if (a->chunk < 0) return RACE_ERR_INVALID_ARG;
+  if (a->grad_dtype != RACE_BF16 && a->grad_dtype != RACE_FP32) return RACE_ERR_INVALID_ARG;
+  if (a->chunk < 0 || a->chunk % 32 != 0) return RACE_ERR_INVALID_ARG;
   if ((double)a->N * a->H * a->d > 4.0e18) return RACE_ERR_INVALID_ARG;
   if (a->d != kD) return RACE_ERR_UNSUPPORTED;
   return RACE_OK;
@@ -269,10 +302,10 @@ race_status_t simt_forward(const race_args_t* a, const T* q, const T* k, const T
   return RACE_OK;
 }
 
-template <typename T, typename TO>
+template <typename T, typename TO, typename TG>
 race_status_t simt_backward(const race_args_t* a, const T* q, const T* k, const T* v,
-                            const float* W, const TO* out, const T* dout, T* dq, T* dk,
-                            T* dv, float* dW, char* ws, cudaStream_t s) {
+                            const float* W, const TO* out, const T* dout, TG* dq, TG* dk,
+                            TG* dv, float* dW, char* ws, cudaStream_t s) {
   SimtPlan p = simt_plan(a, true);
   const Dims& dm = p.dm;
   const int64_t rows = (int64_t)a->H * a->N;
@@ -335,15 +368,15 @@ race_status_t simt_backward(const race_args_t* a, const T* q, const T* k, const 
   RACE_CU(cudaGetLastError());
   {
     RACE_LAUNCH("simt_bwd_finalize_dx", s);
-    simt::k_finalize_dx<T><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(q, dxq, dq, rows);
+    simt::k_finalize_dx<T, TG><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(q, dxq, dq, rows);
   }
   {
     RACE_LAUNCH("simt_bwd_finalize_dx", s);
-    simt::k_finalize_dx<T><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(k, dxk, dk, rows);
+    simt::k_finalize_dx<T, TG><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(k, dxk, dk, rows);
   }
   {
     RACE_LAUNCH("simt_bwd_convert_dv", s);
-    simt::k_convert<T><<<1184, 256, 0, s>>>(dva, dv, rows * kD);
+    simt::k_convert<TG><<<1184, 256, 0, s>>>(dva, dv, rows * kD);
   }
   const int nW = a->L * kD * a->P;
   {
@@ -381,7 +414,7 @@ template <int P>
 race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
                         const CUtensorMap& tk, const CUtensorMap& tv, const float* W,
                         const float* init, float* seg, float* num, const float* inv_norms,
-                        int64_t inv_stride, cudaStream_t s) {
+                        int64_t inv_stride, const float* kscale, cudaStream_t s) {
   dim3 grid(prm.G, prm.n_rg, prm.H);
   const size_t smem = tc::Smem::alloc;
 #define RACE_TC(MODE, NAME)                                                        \
@@ -389,7 +422,7 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
     RACE_CU(set_smem(tc::k_sketch<P, MODE>, smem));                                \
     RACE_LAUNCH(NAME, s);                                                          \
     tc::k_sketch<P, MODE><<<grid, tc::kThreads, smem, s>>>(tq, tk, tv, W, init, seg, \
-                                                            num, prm);             \
+                                                            num, kscale, prm);     \
   } while (0)
   if (mode == tc::kSweep && P == 8 && prm.rows == 256 && inv_norms) {
     CUtensorMap tnum;
@@ -397,13 +430,13 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
     RACE_CU(set_smem(tc::k_sweep_pipe, tc::SPSmem::alloc));
     RACE_LAUNCH("tc_causal_sweep", s);
     tc::k_sweep_pipe<<<grid, tc::kSPThreads, tc::SPSmem::alloc, s>>>(
-        tq, tk, tv, W, init, inv_norms, inv_stride, tnum, num, prm);
+        tq, tk, tv, W, init, inv_norms, inv_stride, tnum, num, kscale, prm);
   } else if (mode == tc::kSweep && prm.rows == 256) {
     constexpr int TABLES = 256 >> P;
     RACE_CU(set_smem(tc::k_sweep<P, TABLES>, tc::SwSmem::alloc));
     RACE_LAUNCH("tc_causal_sweep", s);
     tc::k_sweep<P, TABLES><<<grid, tc::kSwThreads, tc::SwSmem::alloc, s>>>(tq, tk, tv, W, init,
-                                                                          num, prm);
+                                                                          num, kscale, prm);
   } else if (mode == tc::kSweep) RACE_TC(tc::kSweep, "tc_causal_sweep_rows128");
   else if (mode == tc::kBuild) RACE_TC(tc::kBuild, "tc_sketch_build");
   else RACE_TC(tc::kReadout, "tc_readout");
@@ -414,20 +447,23 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
 
 race_status_t tc_dispatch(int P, int mode, const tc::Params& prm, const CUtensorMap& tq,
                           const CUtensorMap& tk, const CUtensorMap& tv, const float* W,
-                          const float* init, float* seg, float* num, cudaStream_t s,
-                          const float* inv_norms = nullptr, int64_t inv_stride = 0) {
+                          const float* init, float* seg, float* num, const float* kscale,
+                          cudaStream_t s, const float* inv_norms = nullptr,
+                          int64_t inv_stride = 0) {
   switch (P) {
-    case 6: return tc_launch<6>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, s);
-    case 7: return tc_launch<7>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, s);
-    case 8: return tc_launch<8>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, s);
+    case 6: return tc_launch<6>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, kscale, s);
+    case 7: return tc_launch<7>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, kscale, s);
+    case 8: return tc_launch<8>(mode, prm, tq, tk, tv, W, init, seg, num, inv_norms, inv_stride, kscale, s);
   }
   return RACE_ERR_UNSUPPORTED;
 }
 
 // Forward accumulators num[h][n][0..64] (unnormalised, den' in column 64) in the
-// forward plan's scratch.
+// forward plan's scratch.  kscale (nullable, [H][N] float32) multiplies every p(k_n):
+// the backward's dv pass runs this with the keys' 1/den'.
 race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k, const void* v,
-                             const float* W, char* ws, float** num_out, cudaStream_t s) {
+                             const float* W, char* ws, float** num_out, cudaStream_t s,
+                             const float* kscale = nullptr) {
   tc::Plan pl = tc::make_plan(a);
   CUtensorMap tq, tk, tv;
   if (!tc::encode_tmap(&tq, q, a->N, a->H) || !tc::encode_tmap(&tk, k, a->N, a->H) ||
@@ -441,7 +477,7 @@ race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k,
   tc::Params prm = pl.prm;
   race_status_t st;
   if (!a->causal || prm.G > 1) {
-    st = tc_dispatch(pl.P, tc::kBuild, prm, tq, tk, tv, W, init, seg, num, s);
+    st = tc_dispatch(pl.P, tc::kBuild, prm, tq, tk, tv, W, init, seg, num, kscale, s);
     if (st != RACE_OK) return st;
     const int RD = prm.rows * tc::kNV;
     {
@@ -462,7 +498,7 @@ race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k,
   }
   RACE_CU(cudaGetLastError());
   st = tc_dispatch(pl.P, a->causal ? tc::kSweep : tc::kReadout, prm, tq, tk, tv, W, init,
-                   seg, num, s, inv_norms, pl.inv_stride);
+                   seg, num, kscale, s, inv_norms, pl.inv_stride);
   if (st != RACE_OK) return st;
   *num_out = num;
   return RACE_OK;
@@ -494,8 +530,8 @@ bool tc_backward_supported(const race_args_t* a) {
 struct BwPlan {
   tc::Params prm;
   int fin_blocks;
-  size_t off_fwd, off_gh, off_gdot, off_rq, off_rk, off_rg, off_duq, off_duk, off_seg,
-      off_init, off_part, bytes;
+  size_t off_fwd, off_rinv, off_gdot, off_rq, off_rk, off_rg, off_rr, off_duq, off_duk,
+      off_seg, off_init, off_part, bytes;
 };
 
 BwPlan make_bw_plan(const race_args_t* a) {
@@ -520,21 +556,26 @@ BwPlan make_bw_plan(const race_args_t* a) {
   p.have_init = 0;
   const int64_t rows = (int64_t)a->H * a->N;
   const int LP = a->L * a->P;
-  b.fin_blocks = (int)std::max<int64_t>(1, std::min<int64_t>(4 * kPlanSMs, (rows + tc::kFinTok - 1) / tc::kFinTok));
+  p.lps = (LP + 7) / 8 * 8;   // 16-byte rows of bf16 per-plane gradients
+  b.fin_blocks = LP <= tc::kFzMaxLP
+                     ? (int)std::max<int64_t>(1, std::min<int64_t>(kPlanSMs, (rows + 127) / 128))
+                     : (int)std::max<int64_t>(1, std::min<int64_t>(4 * kPlanSMs, (rows + tc::kFinTok - 1) / tc::kFinTok));
   const size_t st = (size_t)a->H * p.n_rg * p.G * 256 * tc::kNV * sizeof(float);
   const size_t xb = (size_t)rows * kD * sizeof(__nv_bfloat16);
   size_t o = 0;
   b.off_fwd = o;  o = align_up(o + tc::forward_workspace(a));
-  b.off_gh = o;   o = align_up(o + xb);
+  b.off_rinv = o; o = align_up(o + (size_t)rows * sizeof(float));
   b.off_gdot = o; o = align_up(o + (size_t)rows * sizeof(float));
-  b.off_rq = b.off_rk = b.off_rg = o;
+  b.off_rq = b.off_rk = b.off_rg = b.off_rr = o;
   if (a->causal) {
     b.off_rq = o; o = align_up(o + xb);
     b.off_rk = o; o = align_up(o + xb);
     b.off_rg = o; o = align_up(o + xb);
+    b.off_rr = o; o = align_up(o + (size_t)rows * sizeof(float));
   }
-  b.off_duq = o;  o = align_up(o + (size_t)rows * LP * sizeof(float));
-  b.off_duk = o;  o = align_up(o + (size_t)rows * LP * sizeof(float));
+  // per-plane gradients du' of each side: bf16 hi array then bf16 lo array, [rows][lps]
+  b.off_duq = o;  o = align_up(o + 2 * (size_t)rows * p.lps * sizeof(__nv_bfloat16));
+  b.off_duk = o;  o = align_up(o + 2 * (size_t)rows * p.lps * sizeof(__nv_bfloat16));
   b.off_seg = o;  o = align_up(o + st);
   b.off_init = o; o = align_up(o + st);
   b.off_part = o; o = align_up(o + 2 * (size_t)b.fin_blocks * LP * kD * sizeof(float));
@@ -547,16 +588,17 @@ size_t bw_plan_bytes(const race_args_t* a) { return make_bw_plan(a).bytes; }
 template <int P>
 race_status_t bw_launch(int mode, bool rev, const tc::Params& prm, const CUtensorMap& xa,
                         const CUtensorMap& xb, const CUtensorMap& fa, const CUtensorMap& fb,
-                        const float* ea, const float* eb, const float* W, const float* init,
-                        float* seg, float* du, const char* name, cudaStream_t s) {
+                        const float* ea, const float* eb, const float* ra, const float* rb,
+                        const float* W, const float* init, float* seg, __nv_bfloat16* du,
+                        const char* name, cudaStream_t s) {
   dim3 grid(prm.G, prm.n_rg, prm.H);
   const size_t smem = tc::BwSmem::alloc;
 #define RACE_BW(MODE, REV)                                                                 \
   do {                                                                                     \
     RACE_CU(set_smem(tc::k_bwd_phi<P, MODE, REV>, smem));                                  \
     RACE_LAUNCH(name, s);                                                                  \
-    tc::k_bwd_phi<P, MODE, REV><<<grid, tc::kBwThreads, smem, s>>>(xa, xb, fa, fb, ea, eb, \
-                                                                   W, init, seg, du, prm); \
+    tc::k_bwd_phi<P, MODE, REV><<<grid, tc::kBwThreads, smem, s>>>(                        \
+        xa, xb, fa, fb, ea, eb, ra, rb, W, init, seg, du, prm);                            \
   } while (0)
   if (mode == tc::kBuild) RACE_BW(tc::kBuild, false);
   else if (mode == tc::kReadout) RACE_BW(tc::kReadout, false);
@@ -570,40 +612,53 @@ race_status_t bw_launch(int mode, bool rev, const tc::Params& prm, const CUtenso
 race_status_t bw_dispatch(int P, int mode, bool rev, const tc::Params& prm,
                           const CUtensorMap& xa, const CUtensorMap& xb, const CUtensorMap& fa,
                           const CUtensorMap& fb, const float* ea, const float* eb,
-                          const float* W, const float* init, float* seg, float* du,
-                          const char* name, cudaStream_t s) {
+                          const float* ra, const float* rb, const float* W, const float* init,
+                          float* seg, __nv_bfloat16* du, const char* name, cudaStream_t s) {
   switch (P) {
-    case 6: return bw_launch<6>(mode, rev, prm, xa, xb, fa, fb, ea, eb, W, init, seg, du, name, s);
-    case 7: return bw_launch<7>(mode, rev, prm, xa, xb, fa, fb, ea, eb, W, init, seg, du, name, s);
-    case 8: return bw_launch<8>(mode, rev, prm, xa, xb, fa, fb, ea, eb, W, init, seg, du, name, s);
+    case 6: return bw_launch<6>(mode, rev, prm, xa, xb, fa, fb, ea, eb, ra, rb, W, init, seg, du, name, s);
+    case 7: return bw_launch<7>(mode, rev, prm, xa, xb, fa, fb, ea, eb, ra, rb, W, init, seg, du, name, s);
+    case 8: return bw_launch<8>(mode, rev, prm, xa, xb, fa, fb, ea, eb, ra, rb, W, init, seg, du, name, s);
   }
   return RACE_ERR_UNSUPPORTED;
 }
 
-template <int MT>
-race_status_t finalize_launch_mt(const __nv_bfloat16* q, const float* duq, const float* W,
-                                 __nv_bfloat16* dq, float* partq, const __nv_bfloat16* k,
-                                 const float* duk, __nv_bfloat16* dk, float* partk,
-                                 int64_t rows, int L, int P, int blocks, size_t fsm,
-                                 cudaStream_t s) {
-  RACE_CU(set_smem(tc::k_bwd_finalize<__nv_bfloat16, MT>, fsm));
+template <int MT, typename TG>
+race_status_t finalize_launch_mt(const __nv_bfloat16* x, const __nv_bfloat16* du,
+                                 const float* W, TG* dx, float* part, int64_t rows, int L,
+                                 int P, int lps, int blocks, size_t fsm, cudaStream_t s) {
+  RACE_CU(set_smem(tc::k_bwd_finalize<__nv_bfloat16, MT, TG>, fsm));
   RACE_LAUNCH("tc_bwd_finalize", s);
-  tc::k_bwd_finalize<__nv_bfloat16, MT><<<blocks, 256, fsm, s>>>(q, duq, W, dq, partq, rows, L, P);
-  tc::k_bwd_finalize<__nv_bfloat16, MT><<<blocks, 256, fsm, s>>>(k, duk, W, dk, partk, rows, L, P);
+  tc::k_bwd_finalize<__nv_bfloat16, MT, TG><<<blocks, 256, fsm, s>>>(x, du, W, dx, part, rows,
+                                                                     L, P, lps);
   RACE_CU(cudaGetLastError());
   return RACE_OK;
 }
 
-// dq, dk and the dW partials for L*P projections (MT = ceil(L*P / 16) <= 16).
-race_status_t finalize_launch(int mt, const __nv_bfloat16* q, const float* duq, const float* W,
-                              __nv_bfloat16* dq, float* partq, const __nv_bfloat16* k,
-                              const float* duk, __nv_bfloat16* dk, float* partk, int64_t rows,
-                              int L, int P, int blocks, size_t fsm, cudaStream_t s) {
-#define RACE_FIN(M)                                                                      \
-  case M:                                                                                \
-    return finalize_launch_mt<M>(q, duq, W, dq, partq, k, duk, dk, partk, rows, L, P, \
-                                 blocks, fsm, s)
-  switch (mt) {
+// dx and the dW partials of one side from its per-plane gradients du' (bf16 hi + lo):
+// on tensor cores for L*P <= 128, else on CUDA cores (MT = ceil(L*P / 16) <= 16).
+template <typename TG>
+race_status_t finalize_side(const __nv_bfloat16* x, const __nv_bfloat16* du, const float* W,
+                            TG* dx, float* part, int64_t rows, int L, int P, int lps,
+                            int blocks, cudaStream_t s) {
+  const int LP = L * P;
+  if (LP <= tc::kFzMaxLP) {
+    CUtensorMap tduh, tdul, tx;
+    if (!tc::encode_rows_bf16(&tduh, du, LP, rows, lps) ||
+        !tc::encode_rows_bf16(&tdul, du + (size_t)rows * lps, LP, rows, lps) ||
+        !tc::encode_tmap(&tx, x, rows, 1))
+      return RACE_ERR_CUDA;
+    RACE_CU(set_smem(tc::k_bwd_finalize_tc<TG>, tc::FzSmem::alloc));
+    RACE_LAUNCH("tc_bwd_finalize", s);
+    tc::k_bwd_finalize_tc<TG><<<blocks, tc::kFzThreads, tc::FzSmem::alloc, s>>>(
+        tduh, tdul, tx, W, dx, part, rows, L, P);
+    RACE_CU(cudaGetLastError());
+    return RACE_OK;
+  }
+  const size_t fsm = tc::finalize_smem(LP);
+#define RACE_FIN(M) \
+  case M:           \
+    return finalize_launch_mt<M, TG>(x, du, W, dx, part, rows, L, P, lps, blocks, fsm, s)
+  switch (tc::finalize_mt(LP)) {
     RACE_FIN(1); RACE_FIN(2); RACE_FIN(3); RACE_FIN(4); RACE_FIN(5); RACE_FIN(6); RACE_FIN(7);
     RACE_FIN(8); RACE_FIN(9); RACE_FIN(10); RACE_FIN(11); RACE_FIN(12); RACE_FIN(13);
     RACE_FIN(14); RACE_FIN(15); RACE_FIN(16);
@@ -612,25 +667,25 @@ race_status_t finalize_launch(int mt, const __nv_bfloat16* q, const float* duq, 
   return RACE_ERR_UNSUPPORTED;
 }
 
-template <typename TO>
+template <typename TO, typename TG>
 race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __nv_bfloat16* k,
                           const __nv_bfloat16* v, const float* W, const TO* out,
-                          const __nv_bfloat16* dout, __nv_bfloat16* dq, __nv_bfloat16* dk,
-                          __nv_bfloat16* dv, float* dW, char* ws, cudaStream_t s) {
+                          const __nv_bfloat16* dout, TG* dq, TG* dk, TG* dv, float* dW,
+                          char* ws, cudaStream_t s) {
   const BwPlan pl = make_bw_plan(a);
   const int64_t rows = (int64_t)a->H * a->N;
   const int LP = a->L * a->P;
   char* fws = ws + pl.off_fwd;
-  auto* gh = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_gh);
+  float* rinv = reinterpret_cast<float*>(ws + pl.off_rinv);
   float* gdot = reinterpret_cast<float*>(ws + pl.off_gdot);
-  float* duq = reinterpret_cast<float*>(ws + pl.off_duq);
-  float* duk = reinterpret_cast<float*>(ws + pl.off_duk);
+  auto* duq = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_duq);
+  auto* duk = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_duk);
   float* seg = reinterpret_cast<float*>(ws + pl.off_seg);
   float* init = reinterpret_cast<float*>(ws + pl.off_init);
   float* partq = reinterpret_cast<float*>(ws + pl.off_part);
   float* partk = partq + (size_t)pl.fin_blocks * LP * kD;
   race_status_t st;
-  // ---- den' (recomputed by a forward when not saved) and g''
+  // ---- den' (recomputed by a forward when not saved), -(g . o) and 1/den'
   float* num = nullptr;
   if (!a->den) {
     st = tc_forward_num(a, q, k, v, W, fws, &num, s);
@@ -639,20 +694,21 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   {
     RACE_LAUNCH("tc_bwd_prep", s);
     tc::k_bwd_prep<__nv_bfloat16, TO><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
-        dout, out, num, a->den, gh, gdot, rows, (float)a->L);
+        dout, out, num, a->den, gdot, rinv, rows, (float)a->L);
   }
   RACE_CU(cudaGetLastError());
+  // g enters the feature tiles exactly as given (bf16 upstream gradient)
   CUtensorMap xq, xk, fv, fg;
   if (!tc::encode_tmap(&xq, q, a->N, a->H) || !tc::encode_tmap(&xk, k, a->N, a->H) ||
-      !tc::encode_feat_tmap(&fv, v, a->N, a->H) || !tc::encode_feat_tmap(&fg, gh, a->N, a->H))
+      !tc::encode_feat_tmap(&fv, v, a->N, a->H) || !tc::encode_feat_tmap(&fg, dout, a->N, a->H))
     return RACE_ERR_CUDA;
   const int mode = a->causal ? tc::kSweep : tc::kReadout;
   const int RD = 256 * tc::kNV;
-  // ---- q side: dP(q) = g'' S^T + mask(g'' [v|1]^T) p(k), S over keys j <= i
+  // ---- q side: dP(q) = r (g' S^T + mask(g' [v|1]^T) p(k)), S over keys j <= i
   tc::Params prm = pl.prm;
   if (!a->causal || prm.G > 1) {
-    st = bw_dispatch(a->P, tc::kBuild, false, prm, xk, xk, fv, fv, nullptr, nullptr, W, init,
-                     seg, nullptr, "tc_bwd_build_k", s);
+    st = bw_dispatch(a->P, tc::kBuild, false, prm, xk, xk, fv, fv, nullptr, nullptr, nullptr,
+                     nullptr, W, init, seg, nullptr, "tc_bwd_build_k", s);
     if (st != RACE_OK) return st;
     {
       RACE_LAUNCH("tc_chunk_scan", s);
@@ -662,14 +718,14 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
     RACE_CU(cudaGetLastError());
     prm.have_init = 1;
   }
-  st = bw_dispatch(a->P, mode, false, prm, xq, xk, fg, fv, gdot, nullptr, W, init, seg, duq,
-                   "tc_bwd_q", s);
+  st = bw_dispatch(a->P, mode, false, prm, xq, xk, fg, fv, gdot, nullptr, rinv, nullptr, W,
+                   init, seg, duq, "tc_bwd_q", s);
   if (st != RACE_OK) return st;
-  // ---- k side: dP(k) = [v|1] T^T + mask([v|1] g''^T) p(q), T over queries i >= j
+  // ---- k side: dP(k) = [v|1] T^T + mask([v|1] g'^T) (r p(q)), T over queries i >= j
   prm = pl.prm;
   if (!a->causal || prm.G > 1) {
-    st = bw_dispatch(a->P, tc::kBuild, false, prm, xq, xq, fg, fg, nullptr, gdot, W, init,
-                     seg, nullptr, "tc_bwd_build_q", s);
+    st = bw_dispatch(a->P, tc::kBuild, false, prm, xq, xq, fg, fg, nullptr, gdot, nullptr,
+                     rinv, W, init, seg, nullptr, "tc_bwd_build_q", s);
     if (st != RACE_OK) return st;
     {
       RACE_LAUNCH("tc_chunk_scan", s);
@@ -679,11 +735,11 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
     RACE_CU(cudaGetLastError());
     prm.have_init = 1;
   }
-  st = bw_dispatch(a->P, mode, a->causal != 0, prm, xk, xq, fv, fg, nullptr, gdot, W, init,
-                   seg, duk, "tc_bwd_k", s);
+  st = bw_dispatch(a->P, mode, a->causal != 0, prm, xk, xq, fv, fg, nullptr, gdot, nullptr,
+                   rinv, W, init, seg, duk, "tc_bwd_k", s);
   if (st != RACE_OK) return st;
-  // ---- dv_j = sum_{i >= j} w_ij g_i/den'_i: the forward sweep with queries k, keys q and
-  //      values g'' (sequence reversed for the causal case)
+  // ---- dv_j = sum_{i >= j} w_ij r_i g_i: the forward sweep with queries k, keys q (each
+  //      p(q_i) scaled by r_i) and values g (sequence reversed for the causal case)
   race_args_t av = *a;
   av.den = nullptr;
   float* vnum = nullptr;
@@ -691,29 +747,31 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
     auto* rq = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_rq);
     auto* rk = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_rk);
     auto* rg = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_rg);
+    float* rr = reinterpret_cast<float*>(ws + pl.off_rr);
     const unsigned blocks = (unsigned)((rows * 8 + 255) / 256);
     {
       RACE_LAUNCH("tc_bwd_reverse", s);
       tc::k_reverse_rows<<<blocks, 256, 0, s>>>(q, rq, a->N, a->H);
       tc::k_reverse_rows<<<blocks, 256, 0, s>>>(k, rk, a->N, a->H);
-      tc::k_reverse_rows<<<blocks, 256, 0, s>>>(gh, rg, a->N, a->H);
+      tc::k_reverse_rows<<<blocks, 256, 0, s>>>(dout, rg, a->N, a->H);
+      tc::k_reverse_vec<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(rinv, rr, a->N, a->H);
     }
     RACE_CU(cudaGetLastError());
-    st = tc_forward_num(&av, rk, rq, rg, W, fws, &vnum, s);
+    st = tc_forward_num(&av, rk, rq, rg, W, fws, &vnum, s, rr);
   } else {
-    st = tc_forward_num(&av, k, q, gh, W, fws, &vnum, s);
+    st = tc_forward_num(&av, k, q, dout, W, fws, &vnum, s, rinv);
   }
   if (st != RACE_OK) return st;
   {
     RACE_LAUNCH("tc_bwd_dv_out", s);
-    tc::k_dv_out<__nv_bfloat16><<<(unsigned)((rows * kD + 255) / 256), 256, 0, s>>>(
+    tc::k_dv_out<TG><<<(unsigned)((rows * kD + 255) / 256), 256, 0, s>>>(
         vnum, dv, a->N, a->H, a->causal);
   }
   RACE_CU(cudaGetLastError());
   // ---- dq, dk through the projections and the normalisation; dW
-  const size_t fsm = tc::finalize_smem(LP);
-  st = finalize_launch(tc::finalize_mt(LP), q, duq, W, dq, partq, k, duk, dk, partk, rows, a->L,
-                       a->P, pl.fin_blocks, fsm, s);
+  st = finalize_side(q, duq, W, dq, partq, rows, a->L, a->P, pl.prm.lps, pl.fin_blocks, s);
+  if (st != RACE_OK) return st;
+  st = finalize_side(k, duk, W, dk, partk, rows, a->L, a->P, pl.prm.lps, pl.fin_blocks, s);
   if (st != RACE_OK) return st;
   const int nW = a->L * kD * a->P;
   {
@@ -807,28 +865,40 @@ race_status_t backward_impl(const void* q, const void* k, const void* v, const f
     auto* kk = static_cast<const __nv_bfloat16*>(k);
     auto* vv = static_cast<const __nv_bfloat16*>(v);
     auto* gg = static_cast<const __nv_bfloat16*>(dout);
-    auto* dqq = static_cast<__nv_bfloat16*>(dq);
-    auto* dkk = static_cast<__nv_bfloat16*>(dk);
-    auto* dvv = static_cast<__nv_bfloat16*>(dv);
-    if (a->out_dtype == RACE_BF16)
-      return tc_backward(a, qq, kk, vv, W, static_cast<const __nv_bfloat16*>(out), gg, dqq,
-                         dkk, dvv, dW, sc.ptr, s);
-    return tc_backward(a, qq, kk, vv, W, static_cast<const float*>(out), gg, dqq, dkk, dvv,
-                       dW, sc.ptr, s);
+#define RACE_TBWD(TO, TG)                                                                 \
+  return tc_backward<TO, TG>(a, qq, kk, vv, W, static_cast<const TO*>(out), gg,          \
+                             static_cast<TG*>(dq), static_cast<TG*>(dk), static_cast<TG*>(dv), \
+                             dW, sc.ptr, s)
+    if (a->out_dtype == RACE_BF16) {
+      if (a->grad_dtype == RACE_BF16) RACE_TBWD(__nv_bfloat16, __nv_bfloat16);
+      RACE_TBWD(__nv_bfloat16, float);
+    }
+    if (a->grad_dtype == RACE_BF16) RACE_TBWD(float, __nv_bfloat16);
+    RACE_TBWD(float, float);
+#undef RACE_TBWD
   }
-#define RACE_BWD(T, TO)                                                                  \
-  return simt_backward<T, TO>(a, static_cast<const T*>(q), static_cast<const T*>(k),     \
-                              static_cast<const T*>(v), W, static_cast<const TO*>(out),  \
-                              static_cast<const T*>(dout), static_cast<T*>(dq),          \
-                              static_cast<T*>(dk), static_cast<T*>(dv), dW, sc.ptr, s)
+#define RACE_BWD(T, TO, TG)                                                                \
+  return simt_backward<T, TO, TG>(a, static_cast<const T*>(q), static_cast<const T*>(k),   \
+                                  static_cast<const T*>(v), W, static_cast<const TO*>(out), \
+                                  static_cast<const T*>(dout), static_cast<TG*>(dq),        \
+                                  static_cast<TG*>(dk), static_cast<TG*>(dv), dW, sc.ptr, s)
+#define RACE_BWD_G(T, TO)                                        \
+  do {                                                           \
+    if (a->grad_dtype == RACE_BF16) RACE_BWD(T, TO, __nv_bfloat16); \
+    RACE_BWD(T, TO, float);                                      \
+  } while (0)
   if (a->dtype == RACE_BF16) {
-    if (a->out_dtype == RACE_BF16) RACE_BWD(__nv_bfloat16, __nv_bfloat16);
-    RACE_BWD(__nv_bfloat16, float);
+    if (a->out_dtype == RACE_BF16) RACE_BWD_G(__nv_bfloat16, __nv_bfloat16);
+    RACE_BWD_G(__nv_bfloat16, float);
   }
-  if (a->out_dtype == RACE_BF16) RACE_BWD(float, __nv_bfloat16);
-  RACE_BWD(float, float);
+  if (a->out_dtype == RACE_BF16) RACE_BWD_G(float, __nv_bfloat16);
+  RACE_BWD_G(float, float);
+#undef RACE_BWD_G
 #undef RACE_BWD
 }
+
+// Result word of race_selftest_wait_timeout (1: every lane of the test kernel gave up).
+__device__ int g_selftest_result = 0;
 
 // ------------------------------------------------------------ allocation-free forward
 // Scratch of race_forward_noalloc.  Some callers cannot allocate device memory at call
@@ -839,30 +909,19 @@ race_status_t backward_impl(const void* q, const void* k, const void* v, const f
 // shared by all calls on that device, so overlapping calls race.
 static __device__ __align__(256) char g_noalloc_scratch[RACE_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-char* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device, looked up once per device
-// (the look-up may load the module there, so it belongs before any stream capture).
+// Device address of g_noalloc_scratch on the current device.  It is looked up on every
+// call (a table look-up once the module is loaded there) rather than cached, so that a
+// device reset or a different context on the same device cannot leave a stale address.
+// The first look-up on a device may load the module there, which is why the first call
+// belongs before any stream capture.
 race_status_t noalloc_scratch(char** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
     cudaGetLastError();
     return RACE_ERR_CUDA;
   }
-  if (dev < 0 || dev >= kMaxDevices) return RACE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) {
-      cudaGetLastError();
-      return RACE_ERR_CUDA;
-    }
-    g_noalloc_ptr[dev] = static_cast<char*>(p);
-  }
-  *out = g_noalloc_ptr[dev];
+  *out = static_cast<char*>(p);
   return RACE_OK;
 }
 
@@ -886,12 +945,14 @@ void race_args_init(race_args_t* a, int64_t N, int H, int d, int L, int P, float
   a->causal = causal;
   a->dtype = RACE_BF16;
   a->out_dtype = RACE_BF16;
+  a->grad_dtype = RACE_BF16;
   a->impl = RACE_IMPL_AUTO;
 }
 
 race_status_t race_forward(const void* q, const void* k, const void* v, const float* W,
                            void* out, int64_t N, int H, int d, int L, int P, float tau,
                            int causal, race_stream_t stream) {
+  NvtxRange r("race_forward");
   race_args_t a;
   race_args_init(&a, N, H, d, L, P, tau, causal);
   return forward_impl(q, k, v, W, out, &a, reinterpret_cast<cudaStream_t>(stream));
@@ -901,6 +962,7 @@ race_status_t race_backward(const void* q, const void* k, const void* v, const f
                             const void* out, const void* dout, void* dq, void* dk,
                             void* dv, float* dW, int64_t N, int H, int d, int L, int P,
                             float tau, int causal, race_stream_t stream) {
+  NvtxRange r("race_backward");
   race_args_t a;
   race_args_init(&a, N, H, d, L, P, tau, causal);
   return backward_impl(q, k, v, W, out, dout, dq, dk, dv, dW, &a,
@@ -909,6 +971,7 @@ race_status_t race_backward(const void* q, const void* k, const void* v, const f
 
 race_status_t race_forward_ex(const void* q, const void* k, const void* v, const float* W,
                               void* out, const race_args_t* a, race_stream_t stream) {
+  NvtxRange r("race_forward_ex");
   return forward_impl(q, k, v, W, out, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -916,6 +979,7 @@ race_status_t race_backward_ex(const void* q, const void* k, const void* v,
                                const float* W, const void* out, const void* dout, void* dq,
                                void* dk, void* dv, float* dW, const race_args_t* a,
                                race_stream_t stream) {
+  NvtxRange r("race_backward_ex");
   return backward_impl(q, k, v, W, out, dout, dq, dk, dv, dW, a,
                        reinterpret_cast<cudaStream_t>(stream));
 }
@@ -923,6 +987,7 @@ race_status_t race_backward_ex(const void* q, const void* k, const void* v,
 race_status_t race_forward_noalloc(const void* q, const void* k, const void* v,
                                    const float* W, void* out, const race_args_t* a,
                                    race_stream_t stream) {
+  NvtxRange r("race_forward_noalloc");
   if (!a) return RACE_ERR_INVALID_ARG;
   race_status_t st = check_args(a);
   if (st != RACE_OK) return st;
@@ -975,6 +1040,26 @@ race_status_t race_hash(const void* x, const float* W, void* phi, const race_arg
   }
 #undef RACE_HASH
   RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+race_status_t race_selftest_wait_timeout(int64_t limit_cycles, int* timed_out,
+                                         race_stream_t stream) {
+  if (timed_out) *timed_out = 0;
+  if (limit_cycles < 1 || limit_cycles > tc::kWaitCycles) return RACE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* res = nullptr;
+  RACE_CU(cudaGetSymbolAddress(reinterpret_cast<void**>(&res), g_selftest_result));
+  RACE_CU(cudaMemsetAsync(res, 0, sizeof(int), s));
+  {
+    RACE_LAUNCH("selftest_wait_timeout", s);
+    tc::k_selftest_wait_timeout<<<1, 32, 0, s>>>((long long)limit_cycles, res);
+  }
+  RACE_CU(cudaGetLastError());
+  int v = 0;
+  RACE_CU(cudaMemcpyAsync(&v, res, sizeof(int), cudaMemcpyDeviceToHost, s));
+  RACE_CU(cudaStreamSynchronize(s));
+  if (timed_out) *timed_out = v;
   return RACE_OK;
 }
 

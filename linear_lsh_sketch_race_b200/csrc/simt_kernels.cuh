@@ -569,9 +569,9 @@ __global__ void __launch_bounds__(NT) k_bwd_kv(const T* __restrict__ q,
 }
 
 // dx = (dxhat - xhat (xhat . dxhat)) / |x|  (dxhat / eps when |x| <= eps); warp per row.
-template <typename T>
+template <typename T, typename TG>
 __global__ void k_finalize_dx(const T* __restrict__ x, const float* __restrict__ dxh,
-                              T* __restrict__ dx, int64_t rows) {
+                              TG* __restrict__ dx, int64_t rows) {
   const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (i >= rows) return;
@@ -582,11 +582,11 @@ __global__ void k_finalize_dx(const T* __restrict__ x, const float* __restrict__
     float inv = 1.f / n;
     float xh0 = x0 * inv, xh1 = x1 * inv;
     float dot = warp_sum(xh0 * d0 + xh1 * d1);
-    dx[i * kD + lane] = from_f<T>((d0 - xh0 * dot) * inv);
-    dx[i * kD + lane + 32] = from_f<T>((d1 - xh1 * dot) * inv);
+    dx[i * kD + lane] = from_f<TG>((d0 - xh0 * dot) * inv);
+    dx[i * kD + lane + 32] = from_f<TG>((d1 - xh1 * dot) * inv);
   } else {
-    dx[i * kD + lane] = from_f<T>(d0 / kEpsNorm);
-    dx[i * kD + lane + 32] = from_f<T>(d1 / kEpsNorm);
+    dx[i * kD + lane] = from_f<TG>(d0 / kEpsNorm);
+    dx[i * kD + lane + 32] = from_f<TG>(d1 / kEpsNorm);
   }
 }
 

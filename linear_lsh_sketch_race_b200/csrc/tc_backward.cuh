@@ -2,17 +2,23 @@
 // (one table at R = 256, 256/R tables below).
 //
 // Notation (kernel units: p = unscaled corner probabilities, den' = L * den):
-//   g''_i = [g_i / den'_i , -(g_i . o_i) / den'_i]       (80 wide: the last entry as a
-//                                                          bf16 hi + lo pair, then zeros)
-//   dw_ij = g''_i . [v_j ; 1]                             (gradient of the weight w_ij)
-//   dP(q_i) = sum_{j <= i} dw_ij p(k_j) = S_i g''_i        S_i = sum_{j <= i} p(k_j)[v_j;1]^T
-//   dP(k_j) = sum_{i >= j} dw_ij p(q_i) = T_j [v_j ; 1]    T_j = sum_{i >= j} p(q_i) g''_i^T
-// Both are the same computation with the roles of the two sides exchanged and the
-// sweep reversed: a side "a" whose corner gradients are wanted, with 80-wide features
-// X, and a side "b" with features Y whose p(b) builds the state:
-//   dP_a = X S^T + mask(X Y^T) p(b),   S += p(b)^T Y
-//   q pass: a = q, X = g'', b = k, Y = [v | 1]; forward order, keys j <= i
-//   k pass: a = k, X = [v | 1], b = q, Y = g''; reverse order, queries i >= j
+//   g'_i  = [g_i , -(g_i . o_i)]                          (80 wide: g_i is the upstream
+//                                                          gradient exactly as given, the
+//                                                          last entry a bf16 hi + lo pair)
+//   r_i   = 1 / den'_i                                    (float32)
+//   dw_ij = r_i g'_i . [v_j ; 1]                          (gradient of the weight w_ij)
+//   dP(q_i) = sum_{j <= i} dw_ij p(k_j) = r_i S_i g'_i     S_i = sum_{j <= i} p(k_j)[v_j;1]^T
+//   dP(k_j) = sum_{i >= j} dw_ij p(q_i) = T_j [v_j ; 1]    T_j = sum_{i >= j} r_i p(q_i) g'_i^T
+// The per-row factor r_i is never applied to g (a bf16 rounding of g / den' would cost
+// up to 2^-8, the bf16 unit roundoff, of every gradient entry): on the q side it scales
+// the per-plane gradients in float32, on the k side it scales p(q_i) before its own
+// bf16 rounding.
+// Both sides are the same computation with the roles exchanged and the sweep reversed:
+// a side "a" whose corner gradients are wanted, with 80-wide features X, and a side "b"
+// with features Y whose p(b), times an optional row factor rb, builds the state:
+//   dP_a = ra (X S^T + mask(X Y^T) p~(b)),   S += p~(b)^T Y,   p~(b) = rb p(b)
+//   q pass: a = q, X = g', ra = r, b = k, Y = [v | 1]; forward order, keys j <= i
+//   k pass: a = k, X = [v | 1], b = q, Y = g', rb = r; reverse order, queries i >= j
 // The soft hash backward then gives, per table and plane ([JA] §2.1 soft
 // bucketization; the softmax over corners factorises into logistic pairs),
 //   du_p = (2/tau) (sum_{b: bit p of b set} p_b dP_b - s_p sum_b p_b dP_b),
@@ -115,10 +121,11 @@ __device__ __forceinline__ void store_state_row_split(uint32_t hi_base, uint32_t
 // write_phi_rows for 256 sketch rows with the loop over groups of four high corners kept
 // rolled (a smaller instruction footprint for the sweep's CUDA-core warps): corner
 // c = 4g + jj has high factor p34[jj] (planes 3-4) times the product over planes 5.. chosen
-// by the bits of g.
+// by the bits of g.  Every value is multiplied by `factor` (0 for tokens past the end)
+// before its bf16 rounding.
 template <int P, int TABLES>
 __device__ __forceinline__ void write_phi_rows_rolled(uint32_t tile, int t, const float* u,
-                                                      float scale, bool valid) {
+                                                      float scale, float factor) {
   constexpr int R = 1 << P;
   constexpr int NG = R / 32;
   const uint32_t base = tile + (t >> 3) * (256 * 16) + (t & 7) * 16;
@@ -133,7 +140,7 @@ __device__ __forceinline__ void write_phi_rows_rolled(uint32_t tile, int t, cons
       lo[b] = ((b & 1) ? sp[0] : sm[0]) * ((b & 2) ? sp[1] : sm[1]) * ((b & 4) ? sp[2] : sm[2]);
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj)
-      p34[jj] = (valid ? 1.f : 0.f) * ((jj & 1) ? sp[3] : sm[3]) * ((jj & 2) ? sp[4] : sm[4]);
+      p34[jj] = factor * ((jj & 1) ? sp[3] : sm[3]) * ((jj & 2) ? sp[4] : sm[4]);
 #pragma unroll 1
     for (int g = 0; g < NG; ++g) {
       float hg = 1.f;
@@ -177,14 +184,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     k_bwd_phi(const __grid_constant__ CUtensorMap txa, const __grid_constant__ CUtensorMap txb,
               const __grid_constant__ CUtensorMap tfa, const __grid_constant__ CUtensorMap tfb,
               const float* __restrict__ ea, const float* __restrict__ eb,
+              const float* __restrict__ ra, const float* __restrict__ rb,
               const float* __restrict__ W, const float* __restrict__ init,
-              float* __restrict__ seg_out, float* __restrict__ du_out, Params prm) {
+              float* __restrict__ seg_out, __nv_bfloat16* __restrict__ du_out, Params prm) {
   constexpr bool HAS_A = MODE != kBuild;      // corner gradients of side a
   constexpr bool HAS_B = MODE != kReadout;    // state built from side b
   constexpr bool CAUSAL = MODE == kSweep;
   constexpr int R = 1 << P;
   constexpr int TABLES = 256 / R;
   constexpr int NP = ((TABLES * P + 15) / 16) * 16;
+  static_assert((TABLES * P) % 2 == 0, "per-plane gradients are stored as bf16 pairs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -421,22 +430,36 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     // ================================================================ CUDA-core warps
     const int t = threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int LP = prm.L * P;
-    // the g'' extra value of this thread's token, one step ahead (a global load); at most
-    // one side is the g'' side (ea or eb non-null), the other is [v | 1]
+    // the g' extra value of this thread's token, one step ahead (a global load); at most
+    // one side is the g' side (ea or eb non-null), the other is [v | 1]
     const float* ex_src = HAS_A && ea ? ea : (HAS_B ? eb : nullptr);
+    // the row factors of both sides, [H][N] float32 (null: 1)
+    const float* ra_src = HAS_A ? ra : nullptr;
+    const float* rb_src = HAS_B ? rb : nullptr;
+    auto row_of = [&](int i) { return s0 + (int64_t)(REV ? nchunks - 1 - i : i) * kC + t; };
     auto load_ex = [&](int i) {
-      const int64_t row = s0 + (int64_t)(REV ? nchunks - 1 - i : i) * kC + t;
+      const int64_t row = row_of(i);
       return (ex_src && row < s1) ? ex_src[(size_t)h * prm.N + row] : 0.f;
     };
+    auto load_rf = [&](const float* src, int i) {
+      const int64_t row = row_of(i);
+      return row < s1 ? (src ? src[(size_t)h * prm.N + row] : 1.f) : 0.f;
+    };
     float ex_next = nchunks > 0 ? load_ex(0) : 0.f;
+    float ra_next = nchunks > 0 ? load_rf(ra_src, 0) : 0.f;
+    float rb_next = nchunks > 0 ? load_rf(rb_src, 0) : 0.f;
     for (int i = 0; i < nchunks; ++i) {
       if (s_abort) break;
       const int c = REV ? nchunks - 1 - i : i;
       const int64_t t0 = s0 + (int64_t)c * kC;
       const bool valid = (t0 + t) < s1;
       const float ex = ex_next;
-      if (i + 1 < nchunks) ex_next = load_ex(i + 1);
+      const float fa = ra_next, fb = rb_next;   // row factors (0 past the end)
+      if (i + 1 < nchunks) {
+        ex_next = load_ex(i + 1);
+        ra_next = load_rf(ra_src, i + 1);
+        rb_next = load_rf(rb_src, i + 1);
+      }
       if (!mbar_wait(bar + kbPROJ, i & 1)) { s_abort = 1; break; }
       if (t == 0) BW_TRACE(i, 10);
       tc_fence_after();
@@ -462,7 +485,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
       if (HAS_B) {
         const float sc = row_inv_norm(sm + BwSmem::xb, t) * prm.two_over_tau;
-        write_phi_rows_rolled<P, TABLES>(sb + BwSmem::phb, t, ub, sc, valid);
+        write_phi_rows_rolled<P, TABLES>(sb + BwSmem::phb, t, ub, sc, fb);
         store_extra_cols(sb + BwSmem::fb, t, ex, eb == nullptr, valid);
       }
       fence_proxy_async();
@@ -555,20 +578,34 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
         if (s_abort) break;
         if (valid) {
-          float* dst = du_out + ((size_t)h * prm.N + t0 + t) * LP + (size_t)l0 * P;
-          float d[TABLES * P];
+          // du' = du / max(|x|, eps) as a bf16 hi + lo pair (about 16 significant bits):
+          // the finalize then multiplies by W and by the unnormalised x tile directly
+          const size_t off = ((size_t)h * prm.N + t0 + t) * prm.lps + (size_t)l0 * P;
+          __nv_bfloat16* dh = du_out + off;
+          __nv_bfloat16* dl = du_out + (size_t)prm.H * prm.N * prm.lps + off;
+          const float sc = prm.two_over_tau * fa * inv_a;
+          uint32_t hp[(TABLES * P) / 2], lp[(TABLES * P) / 2];
 #pragma unroll
-          for (int j = 0; j < TABLES; ++j)
+          for (int e = 0; e < TABLES * P; e += 2) {
+            const int j0 = e / P, p0 = e % P, j1 = (e + 1) / P, p1 = (e + 1) % P;
+            const float d0 = sc * (As[j0 * P + p0] - sp[j0 * P + p0] * Ts[j0]);
+            const float d1 = sc * (As[j1 * P + p1] - sp[j1 * P + p1] * Ts[j1]);
+            hp[e / 2] = pack_bf16(d0, d1);
+            lp[e / 2] = pack_bf16(d0 - __uint_as_float(hp[e / 2] << 16),
+                                  d1 - __uint_as_float(hp[e / 2] & 0xffff0000u));
+          }
+          if ((TABLES * P) % 8 == 0) {   // the slice is then 16-byte aligned
 #pragma unroll
-            for (int p = 0; p < P; ++p)
-              d[j * P + p] = prm.two_over_tau * (As[j * P + p] - sp[j * P + p] * Ts[j]);
-          if ((TABLES * P) % 4 == 0) {   // the row group's slice is then 16-byte aligned
-#pragma unroll
-            for (int e = 0; e < TABLES * P; e += 4)
-              *reinterpret_cast<float4*>(dst + e) = make_float4(d[e], d[e + 1], d[e + 2], d[e + 3]);
+            for (int e = 0; e < (TABLES * P) / 2; e += 4) {
+              *reinterpret_cast<uint4*>(dh + 2 * e) = make_uint4(hp[e], hp[e + 1], hp[e + 2], hp[e + 3]);
+              *reinterpret_cast<uint4*>(dl + 2 * e) = make_uint4(lp[e], lp[e + 1], lp[e + 2], lp[e + 3]);
+            }
           } else {
 #pragma unroll
-            for (int e = 0; e < TABLES * P; ++e) dst[e] = d[e];
+            for (int e = 0; e < (TABLES * P) / 2; ++e) {
+              reinterpret_cast<uint32_t*>(dh)[e] = hp[e];
+              reinterpret_cast<uint32_t*>(dl)[e] = lp[e];
+            }
           }
         }
       }
@@ -612,27 +649,34 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 }
 
 // --------------------------------------------------------------------------- helpers
-// g''_i in bf16 (first 64 columns) and its last column -(g_i . o_i)/den'_i in float32.
-// den' comes from the caller's saved den (times L) or from forward accumulators.
+// Per row of the upstream gradient: gdot_i = -(g_i . o_i) (the extra feature column of
+// g'_i) and r_i = 1/den'_i, both float32 (one warp per row).  den' comes from the
+// caller's saved den (times L) or from forward accumulators.
 template <typename T, typename TO>
 __global__ void k_bwd_prep(const T* __restrict__ dout, const TO* __restrict__ out,
                            const float* __restrict__ num, const float* __restrict__ den_in,
-                           __nv_bfloat16* __restrict__ gh, float* __restrict__ gdot,
-                           int64_t rows, float L) {
+                           float* __restrict__ gdot, float* __restrict__ rinv, int64_t rows,
+                           float L) {
   const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (i >= rows) return;
   const float den = den_in ? den_in[i] * L : num[i * kNumStride + kD];
-  const float inv = 1.0f / den;
   const float g0 = to_f(dout[i * kD + 2 * lane]), g1 = to_f(dout[i * kD + 2 * lane + 1]);
   const float o0 = to_f(out[i * kD + 2 * lane]), o1 = to_f(out[i * kD + 2 * lane + 1]);
-  // -(g . o)/den' from the rounded g/den', so that dw_ij = g''_i . [v_j ; 1] is exactly
-  // sum_c bf16(g_c/den') (v_jc - o_ic): no cancellation error when v_j is close to o_i
-  const __nv_bfloat162 r = __floats2bfloat162_rn(g0 * inv, g1 * inv);
-  const float2 rf = __bfloat1622float2(r);
-  const float c = simt::warp_sum(rf.x * o0 + rf.y * o1);
-  reinterpret_cast<__nv_bfloat162*>(gh + i * kD)[lane] = r;
-  if (lane == 0) gdot[i] = -c;
+  const float c = simt::warp_sum(g0 * o0 + g1 * o1);
+  if (lane == 0) {
+    gdot[i] = -c;
+    rinv[i] = 1.0f / den;
+  }
+}
+
+// dst[h][N-1-n] = src[h][n] for float32 [H][N] rows.
+__global__ void k_reverse_vec(const float* __restrict__ src, float* __restrict__ dst,
+                              int64_t N, int H) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)H * N) return;
+  const int64_t h = e / N, n = e % N;
+  dst[h * N + (N - 1 - n)] = src[e];
 }
 
 // dst[h][N-1-n] = src[h][n] for 64-wide bf16 rows.
@@ -662,38 +706,38 @@ __global__ void k_dv_out(const float* __restrict__ num, T* __restrict__ dv, int6
   dv[e] = from_f<T>(num[src * kNumStride + c]);
 }
 
-// dx from du: dxhat = sum_{l,p} W[l][:][p] du[l*P + p]; dx = (dxhat - xhat (xhat . dxhat))
-// / |x| (dxhat / eps when |x| <= eps).  Also per-block partial sums of
-// dW[l][:][p] = sum_n xhat_n du_n[l*P + p] into part[block][L*P][64].
-// Hash backward, last steps, per token x (a row of q or k) with du = dL/du over the L*P
-// projections: dx^ = W du (projection transpose), dx = (dx^ - x^ (x^ . dx^)) / |x|
-// (normalisation Jacobian), and dW partials x^ du^T summed over the tokens of each block.
+// Hash backward, last steps, per token x (a row of q or k) on CUDA cores, for L * P above
+// what the tensor-core finalize (tc_finalize.cuh) covers.  Input du' = (dL/du)/max(|x|,eps)
+// as bf16 hi + lo arrays [rows][lps]: dxh' = W du' (projection transpose),
+// dx = dxh' - xhat (xhat . dxh') (normalisation Jacobian), and dW partials x du'^T summed
+// over the tokens of each block (x unnormalised: x du' = xhat du).
 // 256 threads, 64 tokens per tile, LP padded to LPP = 16 * MT with zero columns.
-// Register tiles: dx^ as 4 tokens x 4 dims per thread over K = LPP in steps of 4; dW as
+// Register tiles: dxh' as 4 tokens x 4 dims per thread over K = LPP in steps of 4; dW as
 // MT consecutive rows x 4 dims per thread over the 64 tokens of the tile.
 constexpr int kMaxLP = 256;
 constexpr int kFinTok = 64;
-template <typename T, int MT>
+template <typename T, int MT, typename TG>
 __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
-                                                     const float* __restrict__ du,
+                                                     const __nv_bfloat16* __restrict__ du,
                                                      const float* __restrict__ W,
-                                                     T* __restrict__ dx, float* __restrict__ part,
-                                                     int64_t rows, int L, int P) {
+                                                     TG* __restrict__ dx, float* __restrict__ part,
+                                                     int64_t rows, int L, int P, int lps) {
   constexpr int LPP = 16 * MT;
   constexpr int LDS = LPP + 4;          // row stride of the du tile (16-byte aligned rows)
   extern __shared__ float4 fsm4[];
   float* fsm = reinterpret_cast<float*>(fsm4);
   const int LP = L * P;
+  const __nv_bfloat16* du_lo = du + (size_t)rows * lps;
   float* Wt = fsm;                       // [LPP][64]: row lp = plane p of table l
   float* dus = Wt + LPP * 64;            // [64 tokens][LDS]
-  float* xh = dus + kFinTok * LDS;       // [64 tokens][68]: x / |x|
-  float* ninv = xh + kFinTok * 68;       // [64]: 1 / max(|x|, eps), 0 for padding rows
+  float* xs = dus + kFinTok * LDS;       // [64 tokens][68]: x
+  float* ninv = xs + kFinTok * 68;       // [64]: 1 / max(|x|, eps), 0 for padding rows
   const int tid = threadIdx.x;
   for (int e = tid; e < LPP * 64; e += 256) {
     const int lp = e / 64, d = e % 64;
     Wt[e] = lp < LP ? W[((size_t)(lp / P) * 64 + d) * P + (lp % P)] : 0.f;
   }
-  const int tg = tid >> 4, dg = (tid & 15) * 4;   // dx^: tokens tg + 16 i, dims dg..dg+3
+  const int tg = tid >> 4, dg = (tid & 15) * 4;   // dxh': tokens tg + 16 i, dims dg..dg+3
   const int rg = (tid >> 4) * MT;                 // dW: rows rg..rg+MT-1, dims dg..dg+3
   float acc[MT][4];
 #pragma unroll
@@ -706,9 +750,14 @@ __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
     const int ntok = (int)min64(kFinTok, rows - base);
     for (int e = tid; e < kFinTok * LPP; e += 256) {
       const int tt = e / LPP, lp = e % LPP;
-      dus[tt * LDS + lp] = (tt < ntok && lp < LP) ? du[(base + tt) * LP + lp] : 0.f;
+      float val = 0.f;
+      if (tt < ntok && lp < LP) {
+        const size_t o = (size_t)(base + tt) * lps + lp;
+        val = __bfloat162float(du[o]) + __bfloat162float(du_lo[o]);
+      }
+      dus[tt * LDS + lp] = val;
     }
-    {   // x / |x|: 4 threads per token, 16 dims each
+    {   // x and 1/|x|: 4 threads per token, 16 dims each
       const int tok = tid >> 2, qd = (tid & 3) * 16;
       const bool live = tok < ntok;
       float xv[16], ss = 0.f;
@@ -721,11 +770,11 @@ __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
       ss += __shfl_xor_sync(0xffffffffu, ss, 2);
       const float inv = 1.0f / fmaxf(sqrtf(ss), kEpsNorm);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) xh[tok * 68 + qd + e] = xv[e] * inv;
+      for (int e = 0; e < 16; ++e) xs[tok * 68 + qd + e] = xv[e];
       if ((tid & 3) == 0) ninv[tok] = live ? inv : 0.f;
     }
     __syncthreads();
-    // ---- dx^ = W du for tokens tg + 16 i
+    // ---- dxh' = W du' for tokens tg + 16 i
     float dxh[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -750,29 +799,30 @@ __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
         }
       }
     }
-    // ---- dx = (dx^ - x^ (x^ . dx^)) / |x|; the 16 threads of a token are 16 lanes
+    // ---- dx = dxh' - x inv^2 (x . dxh'); the 16 threads of a token are 16 lanes
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int tok = tg + 16 * i;
-      const float4 xv = *reinterpret_cast<const float4*>(xh + tok * 68 + dg);
+      const float4 xv = *reinterpret_cast<const float4*>(xs + tok * 68 + dg);
       float dot = xv.x * dxh[i][0] + xv.y * dxh[i][1] + xv.z * dxh[i][2] + xv.w * dxh[i][3];
       dot += __shfl_xor_sync(0xffffffffu, dot, 1);
       dot += __shfl_xor_sync(0xffffffffu, dot, 2);
       dot += __shfl_xor_sync(0xffffffffu, dot, 4);
       dot += __shfl_xor_sync(0xffffffffu, dot, 8);
       const float inv = ninv[tok];
+      const float f = dot * inv * inv;
       if (tok < ntok) {
-        T* o = dx + (base + tok) * kD + dg;
-        o[0] = from_f<T>((dxh[i][0] - xv.x * dot) * inv);
-        o[1] = from_f<T>((dxh[i][1] - xv.y * dot) * inv);
-        o[2] = from_f<T>((dxh[i][2] - xv.z * dot) * inv);
-        o[3] = from_f<T>((dxh[i][3] - xv.w * dot) * inv);
+        TG* o = dx + (base + tok) * kD + dg;
+        o[0] = from_f<TG>(dxh[i][0] - xv.x * f);
+        o[1] = from_f<TG>(dxh[i][1] - xv.y * f);
+        o[2] = from_f<TG>(dxh[i][2] - xv.z * f);
+        o[3] = from_f<TG>(dxh[i][3] - xv.w * f);
       }
     }
     // ---- dW partials: rows rg..rg+MT-1 (table l, plane p), dims dg..dg+3
 #pragma unroll 2
     for (int tt = 0; tt < kFinTok; ++tt) {
-      const float4 xv = *reinterpret_cast<const float4*>(xh + tt * 68 + dg);
+      const float4 xv = *reinterpret_cast<const float4*>(xs + tt * 68 + dg);
       float u[MT];
 #pragma unroll
       for (int m = 0; m < MT; m += 4) {
@@ -827,16 +877,8 @@ __global__ void k_bwd_dw_reduce(const float* __restrict__ pq, const float* __res
 // 3-D view [H][N][64] bf16 of a feature tensor for the 32B-swizzled loads: boxes of
 // 16 columns x 128 rows.
 inline bool encode_feat_tmap(CUtensorMap* m, const void* base, int64_t N, int H) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* f = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !f)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+  const auto fn = tensor_map_encoder();
+  if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)H};
   cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
   cuuint32_t box[3] = {16, (cuuint32_t)kC, 1};

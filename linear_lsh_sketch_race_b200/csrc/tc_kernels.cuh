@@ -19,7 +19,8 @@
 //            S -> bf16 copy in shared memory for the next chunk's readout
 //
 // The same kernel, by MODE, also builds segment sums (no readout) and runs the
-// non-causal readout against a fixed state.  Segments of one sweep start from the
+// non-causal readout against a fixed state.  An optional per-key factor kscale[h][n]
+// multiplies p(k_n) (the backward's dv pass uses the keys' 1/den').  Segments of one sweep start from the
 // exclusive prefix of the segment sums ([JA] §2.2, prefix sums for causal masking).
 #pragma once
 
@@ -50,6 +51,7 @@ struct Params {
   int64_t seg_len;   // tokens per segment (multiple of kC)
   float two_over_tau;
   int have_init;
+  int lps;           // backward: row stride (elements) of the per-plane gradient arrays
 };
 
 // Shared-memory map (bytes from a 1024-aligned base).
@@ -108,10 +110,11 @@ __device__ __forceinline__ void logistic_fast(float z, float& sp, float& sm) {
 // Soft-hash rows of one token for `tables` consecutive tables into the core-matrix
 // tile at `tile` (K-major, no swizzle: core (token/8, row/8) at
 // (token/8)*rows*16 + (row/8)*128, token row within it at (token%8)*16).
-// u[j*P + p] are the raw projections x.W of table j, plane p.
+// u[j*P + p] are the raw projections x.W of table j, plane p; every value is multiplied
+// by `factor` (0 for tokens past the end) before its bf16 rounding.
 template <int P>
 __device__ __forceinline__ void write_phi_rows(uint32_t tile, int t, int rows, int tables,
-                                               const float* u, float scale, bool valid) {
+                                               const float* u, float scale, float factor) {
   constexpr int R = 1 << P;
   constexpr int NHI = R / 8;
   const uint32_t base = tile + (t >> 3) * (rows * 16) + (t & 7) * 16;
@@ -124,7 +127,7 @@ __device__ __forceinline__ void write_phi_rows(uint32_t tile, int t, int rows, i
     for (int b = 0; b < 8; ++b)
       lo[b] = ((b & 1) ? sp[0] : sm[0]) * ((b & 2) ? sp[1] : sm[1]) * ((b & 4) ? sp[2] : sm[2]);
     float hi[NHI];
-    hi[0] = valid ? 1.f : 0.f;
+    hi[0] = factor;
     kron_tree<3, P>(hi, sp, sm);
 #pragma unroll
     for (int c = 0; c < NHI; ++c) {
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_sketch(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const float* __restrict__ W,
              const float* __restrict__ init, float* __restrict__ seg_out,
-             float* __restrict__ num, Params prm) {
+             float* __restrict__ num, const float* __restrict__ kscale, Params prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) u[b * 16 + e] = __uint_as_float(r[e]);
         }
-        write_phi_rows<P>(sb + Smem::phq, t, rows, tables, u, sc, valid);
+        write_phi_rows<P>(sb + Smem::phq, t, rows, tables, u, sc, valid ? 1.f : 0.f);
       }
       if (MODE != kReadout) {
         const float sc = row_inv_norm(sm + Smem::k, t) * prm.two_over_tau;
@@ -391,7 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) u[b * 16 + e] = __uint_as_float(r[e]);
         }
-        write_phi_rows<P>(sb + Smem::phk, t, rows, tables, u, sc, valid);
+        const float kf =
+            valid ? (kscale ? kscale[(size_t)h * prm.N + t0 + t] : 1.f) : 0.f;
+        write_phi_rows<P>(sb + Smem::phk, t, rows, tables, u, sc, kf);
       }
       fence_proxy_async();
       tc_fence_before();
@@ -522,17 +527,24 @@ inline Plan make_plan(const race_args_t* a) {
 
 inline size_t forward_workspace(const race_args_t* a) { return make_plan(a).bytes; }
 
-inline bool encode_tmap(CUtensorMap* m, const void* base, int64_t N, int H) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+// cuTensorMapEncodeTiled through the runtime's driver entry-point query, looked up once
+// (a function-local static: initialised thread-safely, never modified afterwards).
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
     cudaDriverEntryPointQueryResult q;
     void* f = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
             cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !f)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+inline bool encode_tmap(CUtensorMap* m, const void* base, int64_t N, int H) {
+  const auto fn = tensor_map_encoder();
+  if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)H};
   cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
   cuuint32_t box[3] = {64, (cuuint32_t)kC, 1};
@@ -546,16 +558,8 @@ inline bool encode_tmap(CUtensorMap* m, const void* base, int64_t N, int H) {
 // 3-D view [H][N][68] of the float32 output accumulators for TMA reductions: boxes of
 // 64 rows x 68 columns, rows beyond N of a head are dropped.
 inline bool encode_num_tmap(CUtensorMap* m, void* base, int64_t N, int H) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* f = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !f)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+  const auto fn = tensor_map_encoder();
+  if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kNumStride, (cuuint64_t)N, (cuuint64_t)H};
   cuuint64_t strides[2] = {(cuuint64_t)kNumStride * 4, (cuuint64_t)N * kNumStride * 4};
   cuuint32_t box[3] = {(cuuint32_t)kNumStride, 64, 1};

@@ -61,20 +61,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Polling loop of mbar_wait, kept out of line so that the many wait sites of a kernel
 // add little code (instruction-cache footprint) for the rarely taken slow path.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+                                            long long limit) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       raise_status(kStatusTimeout);
       return false;
     }
   }
   return true;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity to complete; gives up after `limit`
+// SM clock cycles (the kernels use kWaitCycles; the self-test passes a short limit).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity);
+  return mbar_wait_slow(bar, parity, limit);
+}
+
+// Self-test of the failure path (one warp, no TMA copy, no MMA): an mbarrier expecting
+// one arrival that never comes is waited on with a limit of `limit` cycles by every lane.
+// Each lane's wait gives up, raises the timeout bit of the device status flag and the
+// kernel returns; the context stays usable.  *out receives 1 if every lane gave up.
+__global__ void k_selftest_wait_timeout(long long limit, int* out) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const bool done = mbar_wait(&bar, 0, limit);
+  const bool all_gave_up = __all_sync(0xffffffffu, !done);
+  if (threadIdx.x == 0) *out = all_gave_up ? 1 : 0;
 }
 
 // ------------------------------------------------------------------------ TMA

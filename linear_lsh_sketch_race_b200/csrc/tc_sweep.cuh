@@ -155,7 +155,8 @@ template <int P, int TABLES>
 __global__ void __launch_bounds__(kSwThreads, 1)
     k_sweep(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const float* __restrict__ W,
-            const float* __restrict__ init, float* __restrict__ num, Params prm) {
+            const float* __restrict__ init, float* __restrict__ num,
+            const float* __restrict__ kscale, Params prm) {
   constexpr int R = 1 << P;
   constexpr int NPL = TABLES * P;               // planes of the CTA
   constexpr int NP = ((NPL + 15) / 16) * 16;    // projection columns
@@ -366,6 +367,10 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       const uint32_t par = c & 1;
       const int64_t t0 = s0 + (int64_t)c * kC;
       const float valid = (t0 + t) < s1 ? 1.f : 0.f;
+      // factor of the expanded corner probabilities: 0 past the end; on the k side the
+      // optional per-key factor
+      const float fac = (grp && kscale && valid != 0.f) ? kscale[(size_t)h * prm.N + t0 + t]
+                                                       : valid;
       // ---- projections and norms
       [[maybe_unused]] const int eb = 10 + 15 * grp;   // trace events of this group
       if (t == 0) SW_TRACE(c, eb + 0);
@@ -392,14 +397,14 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       if (t == 0) SW_TRACE(c, eb + 2);
       if (c > 0 && !wait(kB_HALF0, par ^ 1)) break;
       if (t == 0) SW_TRACE(c, eb + 3);
-      expand_half<P, TABLES, 0>(ph_tile, t, sp, sm_, valid);
+      expand_half<P, TABLES, 0>(ph_tile, t, sp, sm_, fac);
       fence_proxy_async();
       named_bar(nbar, 128);
       if (t == 0) mbar_arrive(bar + (grp ? kB_PHK0 : kB_PHQ0));
       if (t == 0) SW_TRACE(c, eb + 4);
       if (c > 0 && !wait(kB_HALF1, par ^ 1)) break;
       if (t == 0) SW_TRACE(c, eb + 5);
-      expand_half<P, TABLES, 1>(ph_tile, t, sp, sm_, valid);
+      expand_half<P, TABLES, 1>(ph_tile, t, sp, sm_, fac);
       fence_proxy_async();
       named_bar(nbar, 128);
       if (t == 0) mbar_arrive(bar + (grp ? kB_PHK1 : kB_PHQ1));

@@ -23,7 +23,8 @@
 //   warps 8-11  mask QK(c) and round it to bf16 in place; bf16 copy of S for RO(c+1);
 //   warps 12-15 move NUM rows to the float32 output accumulators (TMA reduce-add).
 // Every producer/consumer pair has its own mbarrier; a producer can be at most one
-// phase ahead of its consumer, so parity waits stay unambiguous.
+// phase ahead of its consumer, so parity waits stay unambiguous.  An optional per-key
+// factor kscale[h][n] multiplies p(k_n) (the backward's dv pass uses the keys' 1/den').
 #pragma once
 
 #include "tc_sweep256.cuh"
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
                  const __grid_constant__ CUtensorMap tv, const float* __restrict__ W,
                  const float* __restrict__ init, const float* __restrict__ inv_norms,
                  int64_t inv_stride, const __grid_constant__ CUtensorMap tnum,
-                 float* __restrict__ num, Params prm) {
+                 float* __restrict__ num, const float* __restrict__ kscale, Params prm) {
   constexpr int P = 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -460,6 +461,11 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     for (int x = 0; x < n; ++x) {
       const uint32_t par = x & 1;
       const bool valid = s0 + (int64_t)x * kC + t < s1;
+      // factor of the corner probabilities: 0 past the end, else the optional per-key
+      // factor (loaded before the waits, so its latency overlaps them)
+      const float kf = valid ? (kscale ? kscale[(size_t)h * prm.N + s0 + (int64_t)x * kC + t]
+                                       : 1.f)
+                             : 0.f;
       if (!wait(sp_KT, par) || !wait(sp_PROJK_FULL, par)) break;
       tc_fence_after();
       uint32_t r[16];
@@ -480,7 +486,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       for (int p = 0; p < P; ++p)
         logistic_fast((__uint_as_float(r[p]) + __uint_as_float(r[8 + p])) * scale, sp[p], smv[p]);
       Corners k;
-      corners_of(sp, smv, valid ? 1.f : 0.f, k);
+      corners_of(sp, smv, kf, k);
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int i = 2 * x + half;

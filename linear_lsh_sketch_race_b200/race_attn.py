@@ -32,7 +32,8 @@ _IMPLS = {"auto": RACE_IMPL_AUTO, "simt": RACE_IMPL_SIMT, "tensor": RACE_IMPL_TE
 EXPORTED = ("race_args_init", "race_forward", "race_backward", "race_forward_ex",
             "race_backward_ex", "race_workspace_size", "race_hash", "race_device_status",
             "race_status_string", "race_version", "race_timing_enable",
-            "race_timing_report", "race_launch_count", "race_forward_noalloc")
+            "race_timing_report", "race_launch_count", "race_forward_noalloc",
+            "race_selftest_wait_timeout")
 
 
 class RaceArgs(ctypes.Structure):
@@ -52,6 +53,7 @@ class RaceArgs(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("den", ctypes.c_void_p),
         ("impl", ctypes.c_int),
+        ("grad_dtype", ctypes.c_int),
     ]
 
 
@@ -84,6 +86,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_workspace_size.argtypes = [pargs, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.race_hash.argtypes = [vp, vp, vp, pargs, vp]
     lib.race_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.race_selftest_wait_timeout.argtypes = [i64, ctypes.POINTER(ctypes.c_int), vp]
     lib.race_status_string.argtypes = [i32]
     lib.race_status_string.restype = ctypes.c_char_p
     lib.race_version.argtypes = []
@@ -95,7 +98,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_launch_count.restype = i64
     for name in ("race_forward", "race_backward", "race_forward_ex", "race_backward_ex",
                  "race_forward_noalloc", "race_workspace_size", "race_hash", "race_device_status",
-                 "race_timing_enable", "race_timing_report"):
+                 "race_timing_enable", "race_timing_report", "race_selftest_wait_timeout"):
         getattr(lib, name).restype = i32
     lib.race_version.restype = i32
     _lib = lib
@@ -190,6 +193,15 @@ def race_device_status(stream=None) -> int:
     return flags.value
 
 
+def race_selftest_wait_timeout(limit_cycles: int, stream=None) -> bool:
+    """Run the bounded-wait self-test kernel; True when its wait gave up (the device
+    status flag is then raised for race_device_status to report)."""
+    out = ctypes.c_int(0)
+    _check(load().race_selftest_wait_timeout(int(limit_cycles), ctypes.byref(out),
+                                             _stream(stream)), "race_selftest_wait_timeout")
+    return bool(out.value)
+
+
 def race_timing_enable(on: bool = True):
     _check(load().race_timing_enable(int(bool(on))), "race_timing_enable")
 
@@ -225,12 +237,13 @@ def _dt(t: torch.dtype) -> int:
 
 
 def make_args(q, W, tau, causal, out_dtype=None, chunk=0, impl="auto", den=None,
-              workspace=None) -> RaceArgs:
+              workspace=None, grad_dtype=None) -> RaceArgs:
     H, N, d = q.shape
     L, dW_, P = W.shape
     a = race_args_init(N, H, d, L, P, tau, int(bool(causal)))
     a.dtype = _dt(q.dtype)
     a.out_dtype = _dt(out_dtype or q.dtype)
+    a.grad_dtype = _dt(grad_dtype or q.dtype)
     a.chunk = int(chunk)
     a.impl = _IMPLS[impl]
     if den is not None:
@@ -255,13 +268,16 @@ def forward(q, k, v, W, tau, causal, out_dtype=None, chunk=0, impl="auto",
 
 
 def backward(q, k, v, W, tau, causal, out, dout, den=None, chunk=0, impl="auto",
-             workspace=None, stream=None, grads=None):
-    """Gradients (dq, dk, dv, dW) of sum(out * dout)."""
+             workspace=None, stream=None, grads=None, grad_dtype=None):
+    """Gradients (dq, dk, dv, dW) of sum(out * dout); dq, dk, dv in grad_dtype (default:
+    the dtype of q), dW in float32."""
+    gdt = grad_dtype or q.dtype
     if grads is None:
-        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
-                 torch.empty_like(W))
+        grads = (torch.empty(q.shape, dtype=gdt, device=q.device),
+                 torch.empty(k.shape, dtype=gdt, device=k.device),
+                 torch.empty(v.shape, dtype=gdt, device=v.device), torch.empty_like(W))
     dq, dk, dv, dW = grads
-    a = make_args(q, W, tau, causal, out.dtype, chunk, impl, den, workspace)
+    a = make_args(q, W, tau, causal, out.dtype, chunk, impl, den, workspace, gdt)
     race_backward_ex(q, k, v, W, out, dout, dq, dk, dv, dW, a, stream)
     return dq, dk, dv, dW
 

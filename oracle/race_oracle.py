@@ -312,6 +312,28 @@ def backward_heads(q, k, v, W, tau, causal, dout, out=None, block: int = 256):
     return dq, dk, dv, dW
 
 
+def partial_sums(q, k, v, W, tau, mask=None, block: int = 256):
+    """Unnormalised sums of the definition over a given set of keys:
+    num_i = sum_j a_ij v_j and den_i = sum_j a_ij, a_ij = phi(q_i).phi(k_j), for every
+    query row q_i and every key row k_j given (mask[i, j] in {0, 1}, when given, drops
+    keys).  Summing the results over a split of the keys and dividing gives o_i of
+    ``direct_forward`` ([JA] §2.1 reconstruction: a weighted mean), which is what lets a
+    long sequence be cut into key ranges that are summed independently.
+    Returns (num [n, d], den [n])."""
+    v = np.asarray(v, dtype=np.float64)
+    fq = phi(q, W, tau)
+    num = np.zeros((len(fq), v.shape[1]))
+    den = np.zeros(len(fq))
+    for s in range(0, len(k), block):
+        e = min(s + block, len(k))
+        A = fq @ phi(k[s:e], W, tau).T
+        if mask is not None:
+            A = A * np.asarray(mask)[:, s:e]
+        num += A @ v[s:e]
+        den += A.sum(axis=1)
+    return num, den
+
+
 def forward_rows(q, k, v, W, tau, causal, rows, block: int = 256):
     """Outputs o_i for selected rows ``rows`` of one head, computed one by one from
     the definition (keys limited to j <= i when causal).  Cost grows with the

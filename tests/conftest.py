@@ -1,3 +1,4 @@
+import multiprocessing
 import os
 import sys
 
@@ -11,3 +12,28 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+@pytest.fixture(scope="session")
+def oracle_pool():
+    """Worker processes for float64 oracle work on the full-size workloads.
+
+    Started with the spawn method (a fork after CUDA has been initialised would hang),
+    one single-threaded worker per host core; the workers import only numpy and the
+    oracle package."""
+    n = max(1, os.cpu_count() or 1)
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS",
+                                            "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"
+    try:
+        pool = multiprocessing.get_context("spawn").Pool(n)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    yield pool
+    pool.close()
+    pool.join()

@@ -76,3 +76,9 @@ def test_roofline_takes_the_dominant_kernel_and_keeps_the_forward_sweep():
     assert roof["kernel"] == "tc_causal_sweep" and fwd is None
     # nothing with known work: no roofline
     assert bench.roofline_lines({"tc_normalize": (2.5, 1)}, WL, PEAKS, "test") == (None, None)
+
+
+def test_reported_chunk_is_the_one_the_kernels_run():
+    assert bench.chunk_ran(WL, "auto") == 128          # tensor-core sweep, 128-token chunks
+    assert bench.chunk_ran(WL, "simt") == 32
+    assert bench.chunk_ran(I.WORKLOADS[I.SMALL], "auto") == 32   # float32: CUDA-core tiles

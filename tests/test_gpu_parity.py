@@ -1,11 +1,13 @@
 """GPU parity: the CUDA library against the float64 oracle on identical seeded inputs.
 
 Tolerances (max over all elements, normalised by max|V| for outputs since outputs
-are convex combinations of V rows, and by max|G_ref| for a gradient G):
-  * float32 path:  1e-5
-  * bf16 inputs on the CUDA-core path (float32 arithmetic): 2e-5
+are convex combinations of V rows, and by max|G_ref| of the same gradient tensor G):
+  * CUDA-core path (float32 arithmetic, float32 outputs and gradients): 1e-5 for the
+    backward; 1e-5 (float32 inputs) and 2e-5 (bf16 inputs) for the forward
   * bf16 inputs on the tensor-core path: 2e-3 (bf16 operands, float32 accumulation)
-The oracle receives the exact values the GPU receives (bf16 inputs upcast).
+The oracle receives the exact values the GPU receives (bf16 inputs upcast).  Where a
+gradient is zero in exact arithmetic (dq, dk and hence dW with a single token: o_0 = v_0
+does not depend on q or k), it is measured against max|dv_ref|, the natural scale.
 """
 import numpy as np
 import pytest
@@ -144,23 +146,40 @@ def _oracle_bwd(wl, x):
 def test_backward_simt_parity(causal, N, dtype):
     wl, x, g = _case(N=N, H=2, L=3, P=4, tau=0.6, causal=causal, dtype=dtype, seed=N + 5,
                      backward=True)
-    out = ra.forward(g["q"], g["k"], g["v"], g["W"], wl.tau, causal,
-                     out_dtype=torch.float32, impl="simt")
-    dq, dk, dv, dW = ra.backward(g["q"], g["k"], g["v"], g["W"], wl.tau, causal, out,
-                                 g["dout"], impl="simt")
+    o, _ = _oracle_fwd(wl, x)
+    out = torch.from_numpy(o).float().to(DEV)
+    grads = ra.backward(g["q"], g["k"], g["v"], g["W"], wl.tau, causal, out, g["dout"],
+                        impl="simt", grad_dtype=torch.float32)
     refs = _oracle_bwd(wl, x)
-    tol = 1e-4 if dtype == "fp32" else 4e-3
-    _check_grads((dq, dk, dv, dW), refs, tol)
+    check_grads(grads, refs, 1e-5, N)
 
 
-def _check_grads(got, refs, tol):
-    """max|dG| <= tol * max|G_ref| per gradient; a gradient that is exactly zero in
-    exact arithmetic (dq, dk at N = 1) is measured against the scale of dv."""
-    gscale = np.abs(refs[2]).max()
+def test_backward_simt_bf16_gradients_are_rounded_float32_gradients():
+    wl, x, g = _case(N=300, causal=True, backward=True, seed=2)
+    out = ra.forward(g["q"], g["k"], g["v"], g["W"], wl.tau, True, out_dtype=torch.float32,
+                     impl="simt")
+    f32 = ra.backward(g["q"], g["k"], g["v"], g["W"], wl.tau, True, out, g["dout"],
+                      impl="simt", grad_dtype=torch.float32)
+    b16 = ra.backward(g["q"], g["k"], g["v"], g["W"], wl.tau, True, out, g["dout"],
+                      impl="simt", grad_dtype=torch.bfloat16)
+    # two runs differ in the order of float32 atomic additions; a bf16 result is the
+    # float32 result of its own run rounded once: within one bf16 ulp (2^-7 relative)
+    for a, b in zip(f32[:3], b16[:3]):
+        assert b.dtype == torch.bfloat16
+        assert ((b.float() - a).abs() <= 2.0 ** -7 * a.abs() + 1e-6 * a.abs().max()).all()
+
+
+def check_grads(got, refs, tol, N):
+    """max|dG - dG_ref| <= tol * max|dG_ref| per gradient tensor.  With one token, dq, dk
+    and dW are zero in exact arithmetic and are measured against max|dv_ref|."""
+    errs = {}
     for name, g, ref in zip(("dq", "dk", "dv", "dW"), got, refs):
-        denom = max(np.abs(ref).max(), 0.1 * gscale)
-        err = np.abs(_np(g) - ref).max() / denom
-        assert err <= tol, (name, err)
+        denom = np.abs(ref).max()
+        if N == 1 and name != "dv":
+            denom = np.abs(refs[2]).max()
+        errs[name] = np.abs(_np(g) - ref).max() / denom
+    assert max(errs.values()) <= tol, errs
+    return errs
 
 
 def test_backward_with_saved_den_matches_recompute():
@@ -172,4 +191,4 @@ def test_backward_with_saved_den_matches_recompute():
     b = ra.backward(g["q"], g["k"], g["v"], g["W"], wl.tau, True, out, g["dout"],
                     den=den, impl="simt")
     for x1, x2 in zip(a, b):
-        assert (x1 - x2).abs().max().item() <= 1e-4 * x1.abs().max().item()
+        assert (x1 - x2).abs().max().item() <= 1e-5 * x1.abs().max().item()

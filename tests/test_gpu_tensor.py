@@ -6,12 +6,12 @@ criterion of the method's evaluation.  Shapes cover one and several row groups,
 one and several segments (multi-segment causal sweeps start from scanned segment
 sums), ragged tails and the 128-token chunk edges.
 
-One case uses a looser, derived bound (TOL_FEW): with only L <= 3 tables and a sharp
-kernel (tau = 0.25, P = 8) the estimate averages over few tables, and the bf16
-rounding of phi(q), phi(k) and of one of (state, in-chunk weight) each perturb a
-weight a_ij by up to 2^-9 relative; the output error is then bounded by about
-3 * 2^-9 * max|v_j - o_i| <= 6 * 2^-9 * max|V| ~ 1.2e-2 * max|V|.  Observed errors
-sit near 2e-3; the test allows 4e-3.
+One case uses a looser bound (TOL_FEW): with only L <= 3 tables and a sharp kernel
+(tau = 0.25, P = 8) the estimate averages over few tables, and the bf16 roundings (unit
+roundoff 2^-8) of phi(q), phi(k) and of one of (state, in-chunk weight) each perturb a
+weight a_ij by up to 2^-8 relative; the output error is then at most about
+3 * 2^-8 * max|v_j - o_i| <= 6 * 2^-8 * max|V| ~ 2.3e-2 * max|V|.  Observed errors sit
+near 2e-3; the test allows 4e-3.
 """
 import numpy as np
 import pytest
@@ -120,11 +120,36 @@ def _oracle_rows(wl, x, head, rows):
                                np.asarray(rows))
 
 
-def test_tensor_headline_4m_causal_sampled_rows_and_properties():
+def _oracle_tail_rows(pool, wl, x, head, n_rows):
+    """Causal outputs of the last n_rows rows of one head from the definition: the keys
+    are cut into ranges whose unnormalised sums (oracle.partial_sums) the host cores
+    compute in parallel; the range that overlaps the rows carries the causal mask."""
+    N = wl.N
+    r0 = N - n_rows
+    rows = np.arange(r0, N)
+    qr = x["q"][head, r0:].double().cpu().numpy()
+    kh = x["k"][head].float().cpu().numpy()        # exact: the inputs are bf16
+    vh = x["v"][head].float().cpu().numpy()
+    W = x["W"].double().cpu().numpy()
+    span = 65536
+    tasks = [(qr, kh[s:min(s + span, r0)], vh[s:min(s + span, r0)], W, wl.tau, None)
+             for s in range(0, r0, span)]
+    mask = (np.arange(r0, N)[None, :] <= rows[:, None]).astype(np.float64)
+    tasks.append((qr, kh[r0:], vh[r0:], W, wl.tau, mask))
+    num = np.zeros((n_rows, wl.d))
+    den = np.zeros(n_rows)
+    for a, b in pool.starmap(oracle.partial_sums, tasks, chunksize=1):
+        num += a
+        den += b
+    return num / den[:, None]
+
+
+def test_tensor_headline_4m_causal_rows_and_properties(oracle_pool):
     """The causal 4M-token workload (8 heads, L = 16, P = 8, tau = 0.25) in the launch
-    configuration the benchmark times.  Rows the oracle can compute one by one are
-    compared exactly; every row is checked for convexity and a prefix run for
-    causality."""
+    configuration the benchmark times.  Compared element by element with the oracle:
+    rows at the start (chunk and segment edges) and the last 256 rows of two heads,
+    whose state has absorbed every earlier key; every row is checked for convexity and a
+    prefix run for causality."""
     name = "causal_bf16_h8_n4194304_d64_L16_P8_clustered256"
     wl, x = _full(name)
     q, k, v, W = x["q"], x["k"], x["v"], x["W"]
@@ -140,6 +165,10 @@ def test_tensor_headline_4m_causal_sampled_rows_and_properties():
         ref, _ = _oracle_rows(wl, x, head, rows)
         got = out[head, rows].double().cpu().numpy()
         assert np.abs(got - ref).max() / vmax <= TOL, head
+    for head in (3, 7):
+        ref = _oracle_tail_rows(oracle_pool, wl, x, head, 256)
+        got = out[head, wl.N - 256:].double().cpu().numpy()
+        assert np.abs(got - ref).max() / vmax <= TOL, head
     # convexity: every o_i lies within the running column range of v_0..v_i
     for head in range(wl.H):
         vf = v[head].float()
@@ -153,14 +182,20 @@ def test_tensor_headline_4m_causal_sampled_rows_and_properties():
     assert (short - out[:, :Np]).abs().max().item() <= 1e-5 * vmax
 
 
-def test_tensor_noncausal_262k_sampled_rows():
+def test_tensor_noncausal_262k_all_rows_of_two_heads(oracle_pool):
+    """The non-causal throughput workload (2 x 16 heads, N = 262,144, L = 16, P = 6):
+    every output row of two heads against the oracle's sketch form."""
     name = "noncausal_bf16_b2h16_n262144_d64_L16_P6"
     wl, x = _full(name)
     out = ra.forward(x["q"], x["k"], x["v"], x["W"], wl.tau, False, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    assert ra.race_device_status() == 0
     vmax = x["v"].float().abs().max().item()
-    rows = [0, 1, 777, 131072, 262143]
-    for head in (0, 31):
-        ref, _ = _oracle_rows(wl, x, head, rows)
-        got = out[head, rows].double().cpu().numpy()
-        assert np.abs(got - ref).max() / vmax <= TOL, head
+    W = x["W"].double().cpu().numpy()
+    heads = (0, 31)
+    tasks = [(x["q"][h].float().cpu().numpy(), x["k"][h].float().cpu().numpy(),
+              x["v"][h].float().cpu().numpy(), W, wl.tau, False) for h in heads]
+    refs = oracle_pool.starmap(oracle.forward, tasks, chunksize=1)
+    for h, (ref, _) in zip(heads, refs):
+        got = out[h].double().cpu().numpy()
+        assert np.abs(got - ref).max() / vmax <= TOL, h

@@ -200,6 +200,29 @@ def test_blocked_equals_direct(causal, N, block):
     assert np.allclose(o3, o2[rows], rtol=1e-12, atol=1e-12)
 
 
+def test_partial_sums_over_a_key_split_give_the_definition():
+    """Unnormalised sums over disjoint key ranges add up to the O(N^2) definition: their
+    sum divided by the summed mass is o_i, the summed mass is den_i, and a causal mask
+    over the last range reproduces the causal rows."""
+    rng = np.random.default_rng(31)
+    N = 50
+    q, k, v, W = _rand_case(rng, N)
+    for causal in (False, True):
+        o, den = oracle.direct_forward(q, k, v, W, 0.4, causal)
+        rows = np.array([3, 29, 49])
+        num = np.zeros((len(rows), v.shape[1]))
+        mass = np.zeros(len(rows))
+        for s, e in ((0, 17), (17, 18), (18, 50)):
+            mask = (np.arange(s, e)[None, :] <= rows[:, None]) if causal else None
+            a, b = oracle.partial_sums(q[rows], k[s:e], v[s:e], W, 0.4, mask, block=4)
+            num += a
+            mass += b
+        assert np.allclose(mass, den[rows], rtol=1e-12)
+        assert np.allclose(num / mass[:, None], o[rows], rtol=1e-12, atol=1e-13)
+        o2, d2 = oracle.forward_rows(q, k, v, W, 0.4, causal, rows)
+        assert np.allclose(num / mass[:, None], o2, rtol=1e-12, atol=1e-13)
+
+
 def test_direct_matches_pure_python_loops():
     """A third route written with scalar loops on a 5-token case."""
     rng = np.random.default_rng(8)
