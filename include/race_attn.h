@@ -26,8 +26,9 @@
  *     J(i) = all j (non-causal) or j <= i (causal, inclusive).
  *
  * Layouts.  q, k, v, out, dout, dq, dk, dv are dense row-major [H][N][d] with
- * H = batch * heads (W is shared by every head).  W and dW are dense [L][d][P]
- * float32.  den is [H][N] float32.  phi dumps are [H][N][L*R].
+ * H = batch * heads.  W and dW are dense float32, [L][d][P] shared by every head (the
+ * spec-form calls), or [H][L][d][P] with one set of planes per head (race_args_t
+ * .w_per_head).  den is [H][N] float32.  phi dumps are [H][N][L*R].
  *
  * Pointers.  Every tensor pointer is a DEVICE pointer on the current CUDA device,
  * except where an entry point says "host".  Tensor pointers must be 16-byte aligned.
@@ -101,6 +102,9 @@ typedef struct {
   race_dtype_t grad_dtype;   /* element type of dq, dk, dv written by the backward      */
                              /* (bf16 or float32, for either input dtype; float32 keeps */
                              /* the gradients free of a final bf16 rounding)            */
+  int w_per_head;            /* 0: W and dW are [L][d][P], shared by every head (dW the */
+                             /* sum over heads); 1: W and dW are [H][L][d][P], one set  */
+                             /* of hash planes per head                                 */
 } race_args_t;
 
 /* Fill `a` with the defaults of the spec-form calls: bf16 in, out and gradients,
@@ -171,6 +175,31 @@ race_status_t race_backward_ex(const void *q, const void *k, const void *v,
 race_status_t race_forward_noalloc(const void *q, const void *k, const void *v,
                                    const float *W, void *out, const race_args_t *a,
                                    race_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * race_forward_stream — the forward of race_forward_ex over a block of N new tokens that
+ * continues earlier blocks of the same sequences: every query also attends to all keys of
+ * the earlier blocks through their carried sketch state, which the call updates.  This is
+ * the state carry of decoding (N = 1 per call) and of chunked prefill; the pages name an
+ * efficient KV cache at inference as a use of the sketch ([JA] §6; the state is the
+ * bucket aggregation of [JA] §2.1 and the causal prefix of [JA] §2.2).
+ *
+ * State layout: float32 [H][L * 2^P][65], row l * 2^P + b of head h holding
+ *     sum over earlier keys j of p_{l,b}(k_j) * [v_j | 1]
+ * with p_l = softmax_b(<c_b, W_l^T khat_j>/tau) the unscaled corner probabilities (phi =
+ * p / sqrt(L)): columns 0..63 value sums, column 64 the mass.  (H * L * 2^P * 65 floats;
+ * with per-head planes each head's state uses its own planes.)
+ * state_in: the state before the block (NULL: all zero, the start of a sequence).
+ * state_out: receives the state after the block (NULL: not written); it may be the same
+ * buffer as state_in.  Both must be 16-byte aligned device pointers.
+ * a->causal = 1: keys j <= i within the block plus every earlier key; a->causal = 0: every
+ * key of the block plus every earlier key.  Other arguments, results and errors as
+ * race_forward_ex; the scratch need is race_workspace_size(a, 0).
+ * ------------------------------------------------------------------------------ */
+race_status_t race_forward_stream(const void *q, const void *k, const void *v,
+                                  const float *W, void *out, const float *state_in,
+                                  float *state_out, const race_args_t *a,
+                                  race_stream_t stream);
 
 /* Scratch bytes the *_ex calls need for `a` (backward != 0: the backward).  Writes 0
  * and returns an error status for invalid or unsupported arguments.  Host only; no

@@ -72,6 +72,7 @@ struct Dims {
   int H, L, P, R;
   float tau;
   int causal;
+  int64_t w_hs;   // floats between the hash planes of consecutive heads (0: shared W)
 };
 
 }  // namespace race

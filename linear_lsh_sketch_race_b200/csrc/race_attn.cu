@@ -153,6 +153,7 @@ race_status_t check_args(const race_args_t* a) {
   if (a->impl != RACE_IMPL_AUTO && a->impl != RACE_IMPL_SIMT && a->impl != RACE_IMPL_TENSOR)
     return RACE_ERR_INVALID_ARG;
   if (a->grad_dtype != RACE_BF16 && a->grad_dtype != RACE_FP32) return RACE_ERR_INVALID_ARG;
+  if (a->w_per_head != 0 && a->w_per_head != 1) return RACE_ERR_INVALID_ARG;
   if (a->chunk < 0 || a->chunk % 32 != 0) return RACE_ERR_INVALID_ARG;
   if ((double)a->N * a->H * a->d > 4.0e18) return RACE_ERR_INVALID_ARG;
   if (a->d != kD) return RACE_ERR_UNSUPPORTED;
@@ -168,8 +169,17 @@ Dims dims_of(const race_args_t* a) {
   dm.R = 1 << a->P;
   dm.tau = a->tau;
   dm.causal = a->causal;
+  dm.w_hs = a->w_per_head ? (int64_t)a->L * kD * a->P : 0;
   return dm;
 }
+
+// Carried state of race_forward_stream: the public state [H][L*R][65] the sweep starts
+// from (in, null = zeros) and the state after the call's tokens (out, may be null).
+struct Carry {
+  const float* in = nullptr;
+  float* out = nullptr;
+  bool on = false;
+};
 
 // ----------------------------------------------------------------------------- SIMT
 struct SimtPlan {
@@ -224,7 +234,8 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 // Segment sums and their scan for one side of the sketch (k with [v|1], or q with g'').
 template <typename T, int MODE>
 race_status_t simt_states(const SimtPlan& p, const T* x, const T* v, const float* gpp,
-                          const float* W, char* ws, int scan_mode, cudaStream_t s) {
+                          const float* W, char* ws, int scan_mode, cudaStream_t s,
+                          const Carry* cy = nullptr) {
   const Dims& dm = p.dm;
   simt::Layout ly(dm.R, dm.P);
   float* seg = reinterpret_cast<float*>(ws + p.off_seg);
@@ -239,8 +250,12 @@ race_status_t simt_states(const SimtPlan& p, const T* x, const T* v, const float
   const int RD = dm.R * kDV;
   {
     RACE_LAUNCH("simt_chunk_scan", s);
-    simt::k_scan<<<dim3((RD + 255) / 256, dm.H * dm.L), 256, 0, s>>>(seg, init, RD, p.G,
-                                                                       scan_mode);
+    if (cy && cy->on)
+      simt::k_scan_carry<<<dim3((RD + 255) / 256, dm.H * dm.L), 256, 0, s>>>(
+          seg, init, cy->in, cy->out, dm.R, kDV, dm.L, (int64_t)dm.L * dm.R, p.G, scan_mode);
+    else
+      simt::k_scan<<<dim3((RD + 255) / 256, dm.H * dm.L), 256, 0, s>>>(seg, init, RD, p.G,
+                                                                         scan_mode);
   }
   RACE_CU(cudaGetLastError());
   return RACE_OK;
@@ -248,12 +263,13 @@ race_status_t simt_states(const SimtPlan& p, const T* x, const T* v, const float
 
 template <typename T>
 race_status_t simt_forward_num(const SimtPlan& p, const T* q, const T* k, const T* v,
-                               const float* W, char* ws, cudaStream_t s) {
+                               const float* W, char* ws, cudaStream_t s,
+                               const Carry* cy = nullptr) {
   const Dims& dm = p.dm;
   int have_init = 0;
-  if (!dm.causal || p.G > 1) {
+  if (!dm.causal || p.G > 1 || (cy && cy->on)) {
     race_status_t st =
-        simt_states<T, 0>(p, k, v, nullptr, W, ws, dm.causal ? 0 : 2, s);
+        simt_states<T, 0>(p, k, v, nullptr, W, ws, dm.causal ? 0 : 2, s, cy);
     if (st != RACE_OK) return st;
     have_init = 1;
   }
@@ -289,9 +305,10 @@ void launch_normalize(const float* num, TO* out, float* den, int64_t rows, float
 
 template <typename T, typename TO>
 race_status_t simt_forward(const race_args_t* a, const T* q, const T* k, const T* v,
-                           const float* W, TO* out, char* ws, cudaStream_t s) {
+                           const float* W, TO* out, char* ws, cudaStream_t s,
+                           const Carry* cy = nullptr) {
   SimtPlan p = simt_plan(a, false);
-  race_status_t st = simt_forward_num<T>(p, q, k, v, W, ws, s);
+  race_status_t st = simt_forward_num<T>(p, q, k, v, W, ws, s, cy);
   if (st != RACE_OK) return st;
   const int64_t rows = (int64_t)a->H * a->N;
   {
@@ -378,10 +395,11 @@ race_status_t simt_backward(const race_args_t* a, const T* q, const T* k, const 
     RACE_LAUNCH("simt_bwd_convert_dv", s);
     simt::k_convert<TG><<<1184, 256, 0, s>>>(dva, dv, rows * kD);
   }
-  const int nW = a->L * kD * a->P;
+  const int nW = (a->w_per_head ? a->H : 1) * a->L * kD * a->P;
   {
     RACE_LAUNCH("simt_dW_reduce", s);
-    simt::k_dw_reduce<<<(nW + 255) / 256, 256, 0, s>>>(dwq, dwk, dW, a->H, a->L, p.G, a->P);
+    simt::k_dw_reduce<<<(nW + 255) / 256, 256, 0, s>>>(dwq, dwk, dW, a->H, a->L, p.G, a->P,
+                                                       a->w_per_head);
   }
   RACE_CU(cudaGetLastError());
   return RACE_OK;
@@ -463,7 +481,7 @@ race_status_t tc_dispatch(int P, int mode, const tc::Params& prm, const CUtensor
 // the backward's dv pass runs this with the keys' 1/den'.
 race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k, const void* v,
                              const float* W, char* ws, float** num_out, cudaStream_t s,
-                             const float* kscale = nullptr) {
+                             const float* kscale = nullptr, const Carry* cy = nullptr) {
   tc::Plan pl = tc::make_plan(a);
   CUtensorMap tq, tk, tv;
   if (!tc::encode_tmap(&tq, q, a->N, a->H) || !tc::encode_tmap(&tk, k, a->N, a->H) ||
@@ -476,14 +494,20 @@ race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k,
   RACE_CU(cudaMemsetAsync(num, 0, (size_t)rows * kNumStride * sizeof(float), s));
   tc::Params prm = pl.prm;
   race_status_t st;
-  if (!a->causal || prm.G > 1) {
+  const bool carry = cy && cy->on;
+  if (!a->causal || prm.G > 1 || carry) {
     st = tc_dispatch(pl.P, tc::kBuild, prm, tq, tk, tv, W, init, seg, num, kscale, s);
     if (st != RACE_OK) return st;
     const int RD = prm.rows * tc::kNV;
     {
       RACE_LAUNCH("tc_chunk_scan", s);
-      simt::k_scan<<<dim3((RD + 255) / 256, prm.H * prm.n_rg), 256, 0, s>>>(
-          seg, init, RD, prm.G, a->causal ? 0 : 2);
+      if (carry)
+        simt::k_scan_carry<<<dim3((RD + 255) / 256, prm.H * prm.n_rg), 256, 0, s>>>(
+            seg, init, cy->in, cy->out, prm.rows, tc::kNV, prm.n_rg, (int64_t)prm.L * prm.R,
+            prm.G, a->causal ? 0 : 2);
+      else
+        simt::k_scan<<<dim3((RD + 255) / 256, prm.H * prm.n_rg), 256, 0, s>>>(
+            seg, init, RD, prm.G, a->causal ? 0 : 2);
     }
     RACE_CU(cudaGetLastError());
     prm.have_init = 1;
@@ -506,9 +530,10 @@ race_status_t tc_forward_num(const race_args_t* a, const void* q, const void* k,
 
 template <typename TO>
 race_status_t tc_forward(const race_args_t* a, const void* q, const void* k, const void* v,
-                         const float* W, TO* out, char* ws, cudaStream_t s) {
+                         const float* W, TO* out, char* ws, cudaStream_t s,
+                         const Carry* cy = nullptr) {
   float* num = nullptr;
-  race_status_t st = tc_forward_num(a, q, k, v, W, ws, &num, s);
+  race_status_t st = tc_forward_num(a, q, k, v, W, ws, &num, s, nullptr, cy);
   if (st != RACE_OK) return st;
   const int64_t rows = (int64_t)a->H * a->N;
   {
@@ -557,9 +582,15 @@ BwPlan make_bw_plan(const race_args_t* a) {
   const int64_t rows = (int64_t)a->H * a->N;
   const int LP = a->L * a->P;
   p.lps = (LP + 7) / 8 * 8;   // 16-byte rows of bf16 per-plane gradients
-  b.fin_blocks = LP <= tc::kFzMaxLP
-                     ? (int)std::max<int64_t>(1, std::min<int64_t>(kPlanSMs, (rows + 127) / 128))
-                     : (int)std::max<int64_t>(1, std::min<int64_t>(4 * kPlanSMs, (rows + tc::kFinTok - 1) / tc::kFinTok));
+  p.w_hs = a->w_per_head ? (int64_t)LP * kD : 0;
+  // finalize blocks per head: about one CTA per SM over all heads (tensor-core finalize,
+  // 128-token tiles) or four (CUDA-core finalize, 64-token tiles)
+  {
+    const int tile = LP <= tc::kFzMaxLP ? 128 : tc::kFinTok;
+    const int64_t per_sm = LP <= tc::kFzMaxLP ? 1 : 4;
+    const int64_t want = (per_sm * kPlanSMs + a->H - 1) / a->H;
+    b.fin_blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (a->N + tile - 1) / tile));
+  }
   const size_t st = (size_t)a->H * p.n_rg * p.G * 256 * tc::kNV * sizeof(float);
   const size_t xb = (size_t)rows * kD * sizeof(__nv_bfloat16);
   size_t o = 0;
@@ -578,7 +609,7 @@ BwPlan make_bw_plan(const race_args_t* a) {
   b.off_duk = o;  o = align_up(o + 2 * (size_t)rows * p.lps * sizeof(__nv_bfloat16));
   b.off_seg = o;  o = align_up(o + st);
   b.off_init = o; o = align_up(o + st);
-  b.off_part = o; o = align_up(o + 2 * (size_t)b.fin_blocks * LP * kD * sizeof(float));
+  b.off_part = o; o = align_up(o + 2 * (size_t)a->H * b.fin_blocks * LP * kD * sizeof(float));
   b.bytes = o;
   return b;
 }
@@ -624,40 +655,41 @@ race_status_t bw_dispatch(int P, int mode, bool rev, const tc::Params& prm,
 
 template <int MT, typename TG>
 race_status_t finalize_launch_mt(const __nv_bfloat16* x, const __nv_bfloat16* du,
-                                 const float* W, TG* dx, float* part, int64_t rows, int L,
-                                 int P, int lps, int blocks, size_t fsm, cudaStream_t s) {
+                                 const float* W, TG* dx, float* part, int64_t N, int H, int L,
+                                 int P, int lps, int64_t w_hs, int blocks, size_t fsm,
+                                 cudaStream_t s) {
   RACE_CU(set_smem(tc::k_bwd_finalize<__nv_bfloat16, MT, TG>, fsm));
   RACE_LAUNCH("tc_bwd_finalize", s);
-  tc::k_bwd_finalize<__nv_bfloat16, MT, TG><<<blocks, 256, fsm, s>>>(x, du, W, dx, part, rows,
-                                                                     L, P, lps);
+  tc::k_bwd_finalize<__nv_bfloat16, MT, TG><<<dim3(blocks, H), 256, fsm, s>>>(
+      x, du, W, dx, part, N, L, P, lps, w_hs);
   RACE_CU(cudaGetLastError());
   return RACE_OK;
 }
 
-// dx and the dW partials of one side from its per-plane gradients du' (bf16 hi + lo):
-// on tensor cores for L*P <= 128, else on CUDA cores (MT = ceil(L*P / 16) <= 16).
+// dx and the dW partials [H][blocks][L*P][64] of one side from its per-plane gradients du'
+// (bf16 hi + lo): on tensor cores for L*P <= 128, else on CUDA cores (MT = ceil(L*P/16)).
 template <typename TG>
 race_status_t finalize_side(const __nv_bfloat16* x, const __nv_bfloat16* du, const float* W,
-                            TG* dx, float* part, int64_t rows, int L, int P, int lps,
-                            int blocks, cudaStream_t s) {
+                            TG* dx, float* part, int64_t N, int H, int L, int P, int lps,
+                            int64_t w_hs, int blocks, cudaStream_t s) {
   const int LP = L * P;
   if (LP <= tc::kFzMaxLP) {
     CUtensorMap tduh, tdul, tx;
-    if (!tc::encode_rows_bf16(&tduh, du, LP, rows, lps) ||
-        !tc::encode_rows_bf16(&tdul, du + (size_t)rows * lps, LP, rows, lps) ||
-        !tc::encode_tmap(&tx, x, rows, 1))
+    if (!tc::encode_rows_bf16(&tduh, du, LP, N, H, lps) ||
+        !tc::encode_rows_bf16(&tdul, du + (size_t)H * N * lps, LP, N, H, lps) ||
+        !tc::encode_tmap(&tx, x, N, H))
       return RACE_ERR_CUDA;
     RACE_CU(set_smem(tc::k_bwd_finalize_tc<TG>, tc::FzSmem::alloc));
     RACE_LAUNCH("tc_bwd_finalize", s);
-    tc::k_bwd_finalize_tc<TG><<<blocks, tc::kFzThreads, tc::FzSmem::alloc, s>>>(
-        tduh, tdul, tx, W, dx, part, rows, L, P);
+    tc::k_bwd_finalize_tc<TG><<<dim3(blocks, H), tc::kFzThreads, tc::FzSmem::alloc, s>>>(
+        tduh, tdul, tx, W, dx, part, N, L, P, w_hs);
     RACE_CU(cudaGetLastError());
     return RACE_OK;
   }
   const size_t fsm = tc::finalize_smem(LP);
 #define RACE_FIN(M) \
   case M:           \
-    return finalize_launch_mt<M, TG>(x, du, W, dx, part, rows, L, P, lps, blocks, fsm, s)
+    return finalize_launch_mt<M, TG>(x, du, W, dx, part, N, H, L, P, lps, w_hs, blocks, fsm, s)
   switch (tc::finalize_mt(LP)) {
     RACE_FIN(1); RACE_FIN(2); RACE_FIN(3); RACE_FIN(4); RACE_FIN(5); RACE_FIN(6); RACE_FIN(7);
     RACE_FIN(8); RACE_FIN(9); RACE_FIN(10); RACE_FIN(11); RACE_FIN(12); RACE_FIN(13);
@@ -683,7 +715,7 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   float* seg = reinterpret_cast<float*>(ws + pl.off_seg);
   float* init = reinterpret_cast<float*>(ws + pl.off_init);
   float* partq = reinterpret_cast<float*>(ws + pl.off_part);
-  float* partk = partq + (size_t)pl.fin_blocks * LP * kD;
+  float* partk = partq + (size_t)a->H * pl.fin_blocks * LP * kD;
   race_status_t st;
   // ---- den' (recomputed by a forward when not saved), -(g . o) and 1/den'
   float* num = nullptr;
@@ -769,15 +801,17 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   }
   RACE_CU(cudaGetLastError());
   // ---- dq, dk through the projections and the normalisation; dW
-  st = finalize_side(q, duq, W, dq, partq, rows, a->L, a->P, pl.prm.lps, pl.fin_blocks, s);
+  st = finalize_side(q, duq, W, dq, partq, a->N, a->H, a->L, a->P, pl.prm.lps, pl.prm.w_hs,
+                     pl.fin_blocks, s);
   if (st != RACE_OK) return st;
-  st = finalize_side(k, duk, W, dk, partk, rows, a->L, a->P, pl.prm.lps, pl.fin_blocks, s);
+  st = finalize_side(k, duk, W, dk, partk, a->N, a->H, a->L, a->P, pl.prm.lps, pl.prm.w_hs,
+                     pl.fin_blocks, s);
   if (st != RACE_OK) return st;
-  const int nW = a->L * kD * a->P;
+  const int nW = (a->w_per_head ? a->H : 1) * a->L * kD * a->P;
   {
     RACE_LAUNCH("tc_bwd_dW_reduce", s);
-    tc::k_bwd_dw_reduce<<<(nW + 255) / 256, 256, 0, s>>>(partq, partk, pl.fin_blocks, dW,
-                                                         a->L, a->P);
+    tc::k_bwd_dw_reduce<<<(nW + 255) / 256, 256, 0, s>>>(partq, partk, a->H, pl.fin_blocks,
+                                                         a->w_per_head, dW, a->L, a->P);
   }
   RACE_CU(cudaGetLastError());
   return RACE_OK;
@@ -813,7 +847,8 @@ struct Scratch {
 };
 
 race_status_t forward_impl(const void* q, const void* k, const void* v, const float* W,
-                           void* out, const race_args_t* a, cudaStream_t s) {
+                           void* out, const race_args_t* a, cudaStream_t s,
+                           const Carry* cy = nullptr) {
   race_status_t st = check_args(a);
   if (st != RACE_OK) return st;
   if (!q || !k || !v || !W || !out) return RACE_ERR_INVALID_ARG;
@@ -827,23 +862,23 @@ race_status_t forward_impl(const void* q, const void* k, const void* v, const fl
   if (st != RACE_OK) return st;
   if (tensor) {
     if (a->out_dtype == RACE_BF16)
-      return tc_forward(a, q, k, v, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s);
-    return tc_forward(a, q, k, v, W, static_cast<float*>(out), sc.ptr, s);
+      return tc_forward(a, q, k, v, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s, cy);
+    return tc_forward(a, q, k, v, W, static_cast<float*>(out), sc.ptr, s, cy);
   }
   if (a->dtype == RACE_BF16) {
     auto* qq = static_cast<const __nv_bfloat16*>(q);
     auto* kk = static_cast<const __nv_bfloat16*>(k);
     auto* vv = static_cast<const __nv_bfloat16*>(v);
     if (a->out_dtype == RACE_BF16)
-      return simt_forward(a, qq, kk, vv, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s);
-    return simt_forward(a, qq, kk, vv, W, static_cast<float*>(out), sc.ptr, s);
+      return simt_forward(a, qq, kk, vv, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s, cy);
+    return simt_forward(a, qq, kk, vv, W, static_cast<float*>(out), sc.ptr, s, cy);
   }
   auto* qq = static_cast<const float*>(q);
   auto* kk = static_cast<const float*>(k);
   auto* vv = static_cast<const float*>(v);
   if (a->out_dtype == RACE_BF16)
-    return simt_forward(a, qq, kk, vv, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s);
-  return simt_forward(a, qq, kk, vv, W, static_cast<float*>(out), sc.ptr, s);
+    return simt_forward(a, qq, kk, vv, W, static_cast<__nv_bfloat16*>(out), sc.ptr, s, cy);
+  return simt_forward(a, qq, kk, vv, W, static_cast<float*>(out), sc.ptr, s, cy);
 }
 
 race_status_t backward_impl(const void* q, const void* k, const void* v, const float* W,
@@ -1001,6 +1036,20 @@ race_status_t race_forward_noalloc(const void* q, const void* k, const void* v,
   b.workspace = ws;
   b.workspace_bytes = RACE_NOALLOC_SCRATCH_BYTES;
   return forward_impl(q, k, v, W, out, &b, reinterpret_cast<cudaStream_t>(stream));
+}
+
+race_status_t race_forward_stream(const void* q, const void* k, const void* v,
+                                  const float* W, void* out, const float* state_in,
+                                  float* state_out, const race_args_t* a,
+                                  race_stream_t stream) {
+  NvtxRange r("race_forward_stream");
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+    return RACE_ERR_INVALID_ARG;
+  Carry cy;
+  cy.in = state_in;
+  cy.out = state_out;
+  cy.on = true;
+  return forward_impl(q, k, v, W, out, a, reinterpret_cast<cudaStream_t>(stream), &cy);
 }
 
 race_status_t race_workspace_size(const race_args_t* a, int backward, size_t* bytes) {

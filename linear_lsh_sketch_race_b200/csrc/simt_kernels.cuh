@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(NT) k_hash(const T* __restrict__ x,
   const float scale = rsqrtf((float)dm.L);
   const int LR = dm.L * dm.R;
   for (int l = 0; l < dm.L; ++l) {
-    load_W(W, l, dm.P, sm_ + ly.off_W);
+    load_W(W + (size_t)h * dm.w_hs, l, dm.P, sm_ + ly.off_W);
     __syncthreads();
     tile_soft_hash(xh, tok0, ntok, sm_ + ly.off_W, dm.P, dm.R, 2.f / dm.tau,
                    sm_ + ly.off_xs, sm_ + ly.off_inv, sm_ + ly.off_sp, sm_ + ly.off_sm,
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(NT) k_build(const T* __restrict__ x,
   const int64_t s0 = (int64_t)g * seg_len, s1 = min64(dm.N, s0 + seg_len);
   float* S = sm_ + ly.off_S;
   for (int e = threadIdx.x; e < dm.R * kDV; e += blockDim.x) S[e] = 0.f;
-  load_W(W, l, dm.P, sm_ + ly.off_W);
+  load_W(W + (size_t)h * dm.w_hs, l, dm.P, sm_ + ly.off_W);
   __syncthreads();
   const T* xh = x + (size_t)h * dm.N * kD;
   for (int64_t t0 = s0; t0 < s1; t0 += TT) {
@@ -223,6 +223,39 @@ __global__ void k_scan(const float* __restrict__ seg, float* __restrict__ init, 
   }
 }
 
+// The same prefix with a carried state (streaming): unit u = (head, row group) holds
+// `rows` sketch rows of `ncols` columns (65 used) per segment; carry_in / carry_out are the
+// public state [H][L*R][65] (sketch row = row group * rows + row).  Segment g starts from
+// carry_in plus the sum of segments before it (causal) or from carry_in plus the total
+// (mode 2); carry_out receives carry_in plus the total.  carry_in may be null (zeros) and
+// may equal carry_out (each element is read before it is written, by the same thread).
+__global__ void k_scan_carry(const float* __restrict__ seg, float* __restrict__ init,
+                             const float* carry_in, float* carry_out, int rows, int ncols,
+                             int units_per_head, int64_t LR, int G, int mode) {
+  const int RD = rows * ncols;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= RD) return;
+  const int u = blockIdx.y;
+  const int r = e / ncols, c = e % ncols;
+  const int64_t h = u / units_per_head, rgx = u % units_per_head;
+  const int64_t pub = (h * LR + rgx * rows + r) * kDV + c;
+  const size_t base = (size_t)u * G * RD + e;
+  const float b0 = (c < kDV && carry_in) ? carry_in[pub] : 0.f;
+  float tot = 0.f;
+  for (int g = 0; g < G; ++g) tot += seg[base + (size_t)g * RD];
+  if (mode == 2) {
+    for (int g = 0; g < G; ++g) init[base + (size_t)g * RD] = b0 + tot;
+  } else {
+    float run = b0;
+    for (int g = 0; g < G; ++g) {
+      const float sg = seg[base + (size_t)g * RD];
+      init[base + (size_t)g * RD] = run;
+      run += sg;
+    }
+  }
+  if (c < kDV && carry_out) carry_out[pub] = b0 + tot;
+}
+
 // Start state of a sweep: init[h][l][g] when there is one, else zeros.
 __device__ void load_state(float* S, const float* init, int h, int l, int g, int G,
                            int R, bool have) {
@@ -254,7 +287,7 @@ __global__ void __launch_bounds__(NT) k_fwd_sweep(const T* __restrict__ q,
   float* vals = sm_ + ly.off_vals;
   float* A = sm_ + ly.off_a;
   load_state(S, init, h, l, g, G, R, have_init != 0);
-  load_W(W, l, dm.P, sm_ + ly.off_W);
+  load_W(W + (size_t)h * dm.w_hs, l, dm.P, sm_ + ly.off_W);
   __syncthreads();
   const size_t hoff = (size_t)h * dm.N * kD;
   for (int64_t t0 = s0; t0 < s1; t0 += TT) {
@@ -433,7 +466,7 @@ __global__ void __launch_bounds__(NT) k_bwd_q(const T* __restrict__ q,
   float* spq = sm_ + ly.off_sp;   // q factors stay here: k's hash reuses the x tile only
   float* smq = sm_ + ly.off_sm;
   load_state(S, init, h, l, g, G, R, have_init != 0);
-  load_W(W, l, P, sm_ + ly.off_W);
+  load_W(W + (size_t)h * dm.w_hs, l, P, sm_ + ly.off_W);
   for (int e = threadIdx.x; e < kD * 8; e += blockDim.x) dWs[e] = 0.f;
   __syncthreads();
   const size_t hoff = (size_t)h * dm.N * kD;
@@ -510,7 +543,7 @@ __global__ void __launch_bounds__(NT) k_bwd_kv(const T* __restrict__ q,
   float* spk = sm_ + ly.off_sp;
   float* smk = sm_ + ly.off_sm;
   load_state(S, init, h, l, g, G, R, have_init != 0);
-  load_W(W, l, P, sm_ + ly.off_W);
+  load_W(W + (size_t)h * dm.w_hs, l, P, sm_ + ly.off_W);
   for (int e = threadIdx.x; e < kD * 8; e += blockDim.x) dWs[e] = 0.f;
   __syncthreads();
   const size_t hoff = (size_t)h * dm.N * kD;
@@ -597,15 +630,19 @@ __global__ void k_convert(const float* __restrict__ src, T* __restrict__ dst, in
     dst[i] = from_f<T>(src[i]);
 }
 
-// dW[l][c][p] = sum over heads and segments of both partial buffers, in fixed order.
+// dW[l][c][p] = sum over heads and segments of both partial buffers, in fixed order;
+// with per-head planes dW[h][l][c][p] sums over the segments of head h only.
 __global__ void k_dw_reduce(const float* __restrict__ pq, const float* __restrict__ pk,
-                            float* __restrict__ dW, int H, int L, int G, int P) {
+                            float* __restrict__ dW, int H, int L, int G, int P,
+                            int per_head) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int per = kD * P;
-  if (e >= L * per) return;
-  const int l = e / per, r = e % per;
+  const int n_out = (per_head ? H : 1) * L * per;
+  if (e >= n_out) return;
+  const int hh = e / (L * per), l = (e / per) % L, r = e % per;
+  const int h0 = per_head ? hh : 0, h1 = per_head ? hh + 1 : H;
   float acc = 0.f;
-  for (int h = 0; h < H; ++h)
+  for (int h = h0; h < h1; ++h)
     for (int g = 0; g < G; ++g) {
       size_t o = (((size_t)h * L + l) * G + g) * per + r;
       acc += pq[o] + pk[o];

@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   const int64_t s1 = min64(prm.N, s0 + prm.seg_len);
   const int nchunks = (int)((s1 - s0 + kC - 1) / kC);
   const int l0 = rg * TABLES;
+  W += (size_t)h * prm.w_hs;   // this head's hash planes
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kbCOUNT; ++i) mbar_init(bar + i, 1);
@@ -711,6 +712,8 @@ __global__ void k_dv_out(const float* __restrict__ num, T* __restrict__ dv, int6
 // as bf16 hi + lo arrays [rows][lps]: dxh' = W du' (projection transpose),
 // dx = dxh' - xhat (xhat . dxh') (normalisation Jacobian), and dW partials x du'^T summed
 // over the tokens of each block (x unnormalised: x du' = xhat du).
+// Grid (blocks, H): head h's rows are h*N .. h*N + N - 1 and its planes W + h * w_hs; the
+// partials go to part[h][block][L*P][64].
 // 256 threads, 64 tokens per tile, LP padded to LPP = 16 * MT with zero columns.
 // Register tiles: dxh' as 4 tokens x 4 dims per thread over K = LPP in steps of 4; dW as
 // MT consecutive rows x 4 dims per thread over the 64 tokens of the tile.
@@ -721,13 +724,22 @@ __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
                                                      const __nv_bfloat16* __restrict__ du,
                                                      const float* __restrict__ W,
                                                      TG* __restrict__ dx, float* __restrict__ part,
-                                                     int64_t rows, int L, int P, int lps) {
+                                                     int64_t N, int L, int P, int lps,
+                                                     int64_t w_hs) {
   constexpr int LPP = 16 * MT;
   constexpr int LDS = LPP + 4;          // row stride of the du tile (16-byte aligned rows)
   extern __shared__ float4 fsm4[];
   float* fsm = reinterpret_cast<float*>(fsm4);
   const int LP = L * P;
-  const __nv_bfloat16* du_lo = du + (size_t)rows * lps;
+  const int h = blockIdx.y;
+  const __nv_bfloat16* du_lo = du + (size_t)gridDim.y * N * lps;
+  W += (size_t)h * w_hs;
+  // this head's rows
+  x += (size_t)h * N * kD;
+  du += (size_t)h * N * lps;
+  du_lo += (size_t)h * N * lps;
+  dx += (size_t)h * N * kD;
+  const int64_t rows = N;
   float* Wt = fsm;                       // [LPP][64]: row lp = plane p of table l
   float* dus = Wt + LPP * 64;            // [64 tokens][LDS]
   float* xs = dus + kFinTok * LDS;       // [64 tokens][68]: x
@@ -843,7 +855,7 @@ __global__ void __launch_bounds__(256) k_bwd_finalize(const T* __restrict__ x,
       }
     }
   }
-  float* o = part + (size_t)blockIdx.x * LP * 64;
+  float* o = part + ((size_t)h * gridDim.x + blockIdx.x) * LP * 64;
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     const int lp = rg + m;
@@ -860,17 +872,24 @@ inline size_t finalize_smem(int LP) {
          sizeof(float);
 }
 
-// dW[l][d][p] = sum of the partials of both sides, in fixed order.
+// dW[l][d][p] = sum of the partials [H][blocks][L*P][64] of both sides over heads and
+// blocks, in fixed order; with per-head planes dW[h][l][d][p] sums head h's blocks only.
 __global__ void k_bwd_dw_reduce(const float* __restrict__ pq, const float* __restrict__ pk,
-                                int nblocks, float* __restrict__ dW, int L, int P) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // over L*64*P, W layout
-  if (e >= L * 64 * P) return;
-  const int l = e / (64 * P), d = (e / P) % 64, p = e % P;
+                                int H, int nblocks, int per_head, float* __restrict__ dW,
+                                int L, int P) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // over (H or 1) * L*64*P, W layout
+  const int per = L * 64 * P;
+  if (e >= (per_head ? H : 1) * per) return;
+  const int hh = e / per, r = e % per;
+  const int l = r / (64 * P), d = (r / P) % 64, p = r % P;
   const int LP = L * P;
   const size_t off = (size_t)(l * P + p) * 64 + d;
+  const int h0 = per_head ? hh : 0, h1 = per_head ? hh + 1 : H;
   float acc = 0.f;
-  for (int b = 0; b < nblocks; ++b) acc += pq[(size_t)b * LP * 64 + off];
-  for (int b = 0; b < nblocks; ++b) acc += pk[(size_t)b * LP * 64 + off];
+  for (int h = h0; h < h1; ++h)
+    for (int b = 0; b < nblocks; ++b) acc += pq[((size_t)h * nblocks + b) * LP * 64 + off];
+  for (int h = h0; h < h1; ++h)
+    for (int b = 0; b < nblocks; ++b) acc += pk[((size_t)h * nblocks + b) * LP * 64 + off];
   dW[e] = acc;
 }
 

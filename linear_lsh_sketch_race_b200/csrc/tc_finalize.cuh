@@ -11,10 +11,13 @@
 //   [rows][lps] (about 16 significant bits); W^T is split the same way in shared memory;
 //   x is the bf16 input itself, exact.  dxh' takes three products (hi.hi, lo.hi, hi.lo),
 //   dW two (hi.x, lo.x).
-// One CTA per SM, persistent over tiles of 128 tokens, two TMA stages.  Warps 0-3 (thread
-// = token = tensor-memory lane) compute 1/|x| from the x tile, read dxh' and write dx;
-// warp 4 issues TMA copies and MMAs from an elected lane.  L * P <= 128: one accumulator
-// of 128 lanes holds dW (lane = table * P + plane), and the du' tile is two boxes of 64.
+// Grid (blocks, H): the CTAs of head h are persistent over its tiles of 128 tokens (the
+// tensor maps are [H][N][cols], so a tile never reaches into the next head), two TMA
+// stages.  Warps 0-3 (thread = token = tensor-memory lane) compute 1/|x| from the x tile,
+// read dxh' and write dx; warp 4 issues TMA copies and MMAs from an elected lane.
+// L * P <= 128: one accumulator of 128 lanes holds dW (lane = table * P + plane), and the
+// du' tile is two boxes of 64.  W is this head's planes (offset w_hs per head, 0 when
+// shared); the partial sums go to part[h][block][L*P][64].
 #pragma once
 
 #include "tc_kernels.cuh"
@@ -45,8 +48,8 @@ __global__ void __launch_bounds__(kFzThreads, 1)
     k_bwd_finalize_tc(const __grid_constant__ CUtensorMap tduh,
                       const __grid_constant__ CUtensorMap tdul,
                       const __grid_constant__ CUtensorMap tx, const float* __restrict__ W,
-                      TG* __restrict__ dx, float* __restrict__ part, int64_t rows, int L,
-                      int P) {
+                      TG* __restrict__ dx, float* __restrict__ part, int64_t N, int L,
+                      int P, int64_t w_hs) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -55,7 +58,9 @@ __global__ void __launch_bounds__(kFzThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + fz_COUNT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int LP = L * P;
-  const int64_t ntiles = (rows + 127) / 128;
+  const int h = blockIdx.y;
+  W += (size_t)h * w_hs;
+  const int64_t ntiles = (N + 127) / 128;
   const int my_tiles =
       blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
 
@@ -104,10 +109,10 @@ __global__ void __launch_bounds__(kFzThreads, 1)
       mbar_arrive_expect_tx(bar + fz_FULL0 + st, FzSmem::stage);
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
-        tma_load_3d(sm + base + FzSmem::duh + b * 16384, &tduh, 64 * b, r0, 0, bar + fz_FULL0 + st);
-        tma_load_3d(sm + base + FzSmem::dul + b * 16384, &tdul, 64 * b, r0, 0, bar + fz_FULL0 + st);
+        tma_load_3d(sm + base + FzSmem::duh + b * 16384, &tduh, 64 * b, r0, h, bar + fz_FULL0 + st);
+        tma_load_3d(sm + base + FzSmem::dul + b * 16384, &tdul, 64 * b, r0, h, bar + fz_FULL0 + st);
       }
-      tma_load_3d(sm + base + FzSmem::x, &tx, 0, r0, 0, bar + fz_FULL0 + st);
+      tma_load_3d(sm + base + FzSmem::x, &tx, 0, r0, h, bar + fz_FULL0 + st);
     };
     if (elect_one()) {
       prefetch_tmap(&tduh);
@@ -206,8 +211,8 @@ __global__ void __launch_bounds__(kFzThreads, 1)
       for (int c = 0; c < 64; ++c) dot = fmaf(xr[c], __uint_as_float(r[c]), dot);
       const float f = dot * inv * inv;
       const int64_t row = (int64_t)tile_row0(k) + t;
-      if (row < rows) {
-        TG* o = dx + row * kD;
+      if (row < N) {
+        TG* o = dx + ((size_t)h * N + row) * kD;
         if constexpr (sizeof(TG) == 4) {
 #pragma unroll
           for (int c = 0; c < 64; c += 4)
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(kFzThreads, 1)
         for (int b = 0; b < 4; ++b) tmem_ld16(tmem + lane_off + TM_DW + b * 16, r + b * 16);
         tmem_ld_wait();
         if (t < LP) {
-          float* o = part + ((size_t)blockIdx.x * LP + t) * 64;
+          float* o = part + (((size_t)h * gridDim.x + blockIdx.x) * LP + t) * 64;
 #pragma unroll
           for (int c = 0; c < 64; c += 4)
             *reinterpret_cast<float4*>(o + c) =
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(kFzThreads, 1)
         }
       }
     } else if (t < LP) {
-      float* o = part + ((size_t)blockIdx.x * LP + t) * 64;
+      float* o = part + (((size_t)h * gridDim.x + blockIdx.x) * LP + t) * 64;
       for (int c = 0; c < 64; ++c) o[c] = 0.f;
     }
   }
@@ -262,15 +267,15 @@ __global__ void __launch_bounds__(kFzThreads, 1)
   }
 }
 
-// 2-D bf16 view [rows][inner] with the given row stride, for 128B-swizzled boxes of
-// 64 elements x 128 rows (a 3-D map with a unit outer dimension).
-inline bool encode_rows_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t rows,
+// 3-D bf16 view [H][N][inner] with the given row stride (elements), for 128B-swizzled
+// boxes of 64 elements x 128 rows of one head.
+inline bool encode_rows_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t N, int H,
                              int64_t row_stride_elems) {
   const auto fn = tensor_map_encoder();
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, 1};
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)H};
   cuuint64_t strides[2] = {(cuuint64_t)row_stride_elems * 2,
-                           (cuuint64_t)row_stride_elems * 2 * (cuuint64_t)rows};
+                           (cuuint64_t)row_stride_elems * 2 * (cuuint64_t)N};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,

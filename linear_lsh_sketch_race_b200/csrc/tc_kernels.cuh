@@ -52,6 +52,7 @@ struct Params {
   float two_over_tau;
   int have_init;
   int lps;           // backward: row stride (elements) of the per-plane gradient arrays
+  int64_t w_hs;      // floats between the hash planes of consecutive heads (0: shared W)
 };
 
 // Shared-memory map (bytes from a 1024-aligned base).
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t s1 = min64(prm.N, s0 + prm.seg_len);
   const int nchunks = (int)((s1 - s0 + kC - 1) / kC);
   const int l0 = rg * tables;
+  W += (size_t)h * prm.w_hs;   // this head's hash planes
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
@@ -513,6 +515,8 @@ inline Plan make_plan(const race_args_t* a) {
   p.G = (int)((a->N + p.seg_len - 1) / p.seg_len);
   p.two_over_tau = 2.0f / a->tau;
   p.have_init = 0;
+  p.lps = 0;
+  p.w_hs = a->w_per_head ? (int64_t)a->L * kD * a->P : 0;
   const size_t st = (size_t)a->H * p.n_rg * p.G * p.rows * kNV * sizeof(float);
   size_t o = 0;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };

@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   const int64_t s1 = min64(prm.N, s0 + prm.seg_len);
   const int nchunks = (int)((s1 - s0 + kC - 1) / kC);
   const int l0 = rg * TABLES;
+  W += (size_t)h * prm.w_hs;   // this head's hash planes
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kB_COUNT; ++i)

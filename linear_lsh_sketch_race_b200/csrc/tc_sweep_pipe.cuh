@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   const int64_t s0 = (int64_t)g * prm.seg_len;
   const int64_t s1 = min64(prm.N, s0 + prm.seg_len);
   const int n = (int)((s1 - s0 + kC - 1) / kC);
+  W += (size_t)h * prm.w_hs;   // this head's hash planes
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < sp_COUNT; ++i) {

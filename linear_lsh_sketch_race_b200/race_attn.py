@@ -33,7 +33,7 @@ EXPORTED = ("race_args_init", "race_forward", "race_backward", "race_forward_ex"
             "race_backward_ex", "race_workspace_size", "race_hash", "race_device_status",
             "race_status_string", "race_version", "race_timing_enable",
             "race_timing_report", "race_launch_count", "race_forward_noalloc",
-            "race_selftest_wait_timeout")
+            "race_selftest_wait_timeout", "race_forward_stream")
 
 
 class RaceArgs(ctypes.Structure):
@@ -54,6 +54,7 @@ class RaceArgs(ctypes.Structure):
         ("den", ctypes.c_void_p),
         ("impl", ctypes.c_int),
         ("grad_dtype", ctypes.c_int),
+        ("w_per_head", ctypes.c_int),
     ]
 
 
@@ -83,6 +84,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_forward_ex.argtypes = [vp, vp, vp, vp, vp, pargs, vp]
     lib.race_backward_ex.argtypes = [vp] * 10 + [pargs, vp]
     lib.race_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, pargs, vp]
+    lib.race_forward_stream.argtypes = [vp, vp, vp, vp, vp, vp, vp, pargs, vp]
     lib.race_workspace_size.argtypes = [pargs, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.race_hash.argtypes = [vp, vp, vp, pargs, vp]
     lib.race_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -98,7 +100,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_launch_count.restype = i64
     for name in ("race_forward", "race_backward", "race_forward_ex", "race_backward_ex",
                  "race_forward_noalloc", "race_workspace_size", "race_hash", "race_device_status",
-                 "race_timing_enable", "race_timing_report", "race_selftest_wait_timeout"):
+                 "race_timing_enable", "race_timing_report", "race_selftest_wait_timeout",
+                 "race_forward_stream"):
         getattr(lib, name).restype = i32
     lib.race_version.restype = i32
     _lib = lib
@@ -166,6 +169,12 @@ def race_forward_noalloc(q, k, v, W, out, args: RaceArgs, stream=None):
     _check(load().race_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out),
                                        ctypes.byref(args), _stream(stream)),
            "race_forward_noalloc")
+
+
+def race_forward_stream(q, k, v, W, out, state_in, state_out, args: RaceArgs, stream=None):
+    _check(load().race_forward_stream(_ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out),
+                                      _ptr(state_in), _ptr(state_out), ctypes.byref(args),
+                                      _stream(stream)), "race_forward_stream")
 
 
 def race_backward_ex(q, k, v, W, out, dout, dq, dk, dv, dW, args: RaceArgs, stream=None):
@@ -239,8 +248,14 @@ def _dt(t: torch.dtype) -> int:
 def make_args(q, W, tau, causal, out_dtype=None, chunk=0, impl="auto", den=None,
               workspace=None, grad_dtype=None) -> RaceArgs:
     H, N, d = q.shape
-    L, dW_, P = W.shape
+    if W.dim() == 4:                     # one set of planes per head: [H, L, d, P]
+        if W.shape[0] != H:
+            raise ValueError(f"per-head planes {tuple(W.shape)} for {H} heads")
+        _, L, dW_, P = W.shape
+    else:                                # shared planes: [L, d, P]
+        L, dW_, P = W.shape
     a = race_args_init(N, H, d, L, P, tau, int(bool(causal)))
+    a.w_per_head = int(W.dim() == 4)
     a.dtype = _dt(q.dtype)
     a.out_dtype = _dt(out_dtype or q.dtype)
     a.grad_dtype = _dt(grad_dtype or q.dtype)
@@ -282,10 +297,34 @@ def backward(q, k, v, W, tau, causal, out, dout, den=None, chunk=0, impl="auto",
     return dq, dk, dv, dW
 
 
+def state_shape(H: int, L: int, P: int):
+    """Shape of the carried sketch state of race_forward_stream: [H, L * 2^P, 65]."""
+    return (H, L << P, 65)
+
+
+def forward_stream(q, k, v, W, tau, causal=True, state=None, out_dtype=None, impl="auto",
+                   inplace=False, stream=None):
+    """RACE attention over a block of new tokens that continues earlier blocks: returns
+    (out, new_state).  `state` is the carried [H, L*2^P, 65] float32 state (None: start of
+    the sequences); with inplace=True it is updated in place and returned."""
+    out_dtype = out_dtype or q.dtype
+    out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    H = q.shape[0]
+    L, P = W.shape[-3], W.shape[-1]
+    if inplace and state is not None:
+        new_state = state
+    else:
+        new_state = torch.empty(state_shape(H, L, P), dtype=torch.float32, device=q.device)
+    a = make_args(q, W, tau, causal, out_dtype, 0, impl)
+    race_forward_stream(q, k, v, W, out, state, new_state, a, stream)
+    return out, new_state
+
+
 def hash(x, W, tau, out_dtype=torch.float32, stream=None):  # noqa: A001
-    """phi(x) = concat_l softmax-over-corners / sqrt(L), shape [H, N, L*2^P]."""
+    """phi(x) = concat_l softmax-over-corners / sqrt(L), shape [H, N, L*2^P]; W shared
+    [L, d, P] or per head [H, L, d, P]."""
     H, N, d = x.shape
-    L, _, P = W.shape
+    L, P = W.shape[-3], W.shape[-1]
     phi = torch.empty((H, N, L << P), dtype=out_dtype, device=x.device)
     a = make_args(x, W, tau, False, out_dtype)
     race_hash(x, W, phi, a, stream)

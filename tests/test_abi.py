@@ -43,7 +43,7 @@ int main(void) {
   printf("%zu", sizeof(race_args_t));
 #define F(m) printf(" %zu", offsetof(race_args_t, m));
   F(N) F(H) F(d) F(L) F(P) F(tau) F(causal) F(dtype) F(out_dtype) F(chunk)
-  F(workspace) F(workspace_bytes) F(den) F(impl) F(grad_dtype)
+  F(workspace) F(workspace_bytes) F(den) F(impl) F(grad_dtype) F(w_per_head)
   printf("\n");
   return 0;
 }
@@ -78,7 +78,7 @@ def test_args_init_defaults():
     assert (a.N, a.H, a.d, a.L, a.P, a.causal) == (1024, 2, 64, 4, 4, 1)
     assert a.dtype == ra.RACE_BF16 and a.out_dtype == ra.RACE_BF16
     assert a.impl == ra.RACE_IMPL_AUTO and a.chunk == 0 and not a.workspace and not a.den
-    assert a.grad_dtype == ra.RACE_BF16
+    assert a.grad_dtype == ra.RACE_BF16 and a.w_per_head == 0
 
 
 @pytest.mark.parametrize("field,value,status", [
@@ -97,6 +97,7 @@ def test_args_init_defaults():
     ("chunk", -64, ra.RACE_ERR_INVALID_ARG),
     ("chunk", 100, ra.RACE_ERR_INVALID_ARG),
     ("grad_dtype", 3, ra.RACE_ERR_INVALID_ARG),
+    ("w_per_head", 2, ra.RACE_ERR_INVALID_ARG),
     ("d", 32, ra.RACE_ERR_UNSUPPORTED),
     ("d", 128, ra.RACE_ERR_UNSUPPORTED),
 ])
