@@ -201,6 +201,27 @@ race_status_t race_forward_stream(const void *q, const void *k, const void *v,
                                   float *state_out, const race_args_t *a,
                                   race_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * race_hard_forward — classic RACE with hard hashes, the tau -> 0 limit of the soft
+ * estimator: repeated arrays of counts ([JA] §2.1 count estimators and bucket
+ * aggregation; [KO] §2: L tables of P-bit buckets).  With h_l(x) the P-bit bucket whose
+ * bit p is 1 when W_l[:,p] . x >= 0 (decided in float32),
+ *     A_ij = number of tables l with h_l(q_i) == h_l(k_j)      (j in J(i))
+ *     out_i = sum_j A_ij v_j / sum_j A_ij,  and out_i = 0 when no key collides.
+ * counts (nullable, int32 [H][N], device): receives sum_j A_ij, exact.  tau is ignored;
+ * other arguments and layouts as race_forward_ex (P <= 8).  Scratch as race_forward_ex
+ * with the size given by race_hard_workspace_size.
+ * ------------------------------------------------------------------------------ */
+race_status_t race_hard_forward(const void *q, const void *k, const void *v, const float *W,
+                                void *out, int *counts, const race_args_t *a,
+                                race_stream_t stream);
+race_status_t race_hard_workspace_size(const race_args_t *a, size_t *bytes);
+
+/* race_hard_hash — the bucket ids alone: ids[h][n][l] = h_l(x_hn) as uint8 (device),
+ * for x of a->dtype [H][N][d]. */
+race_status_t race_hard_hash(const void *x, const float *W, uint8_t *ids, const race_args_t *a,
+                             race_stream_t stream);
+
 /* Scratch bytes the *_ex calls need for `a` (backward != 0: the backward).  Writes 0
  * and returns an error status for invalid or unsupported arguments.  Host only; no
  * device work. */

@@ -20,6 +20,7 @@
 #include "tc_sweep_pipe.cuh"
 #include "tc_backward.cuh"
 #include "tc_finalize.cuh"
+#include "hard_kernels.cuh"
 
 namespace race {
 
@@ -817,6 +818,104 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   return RACE_OK;
 }
 
+// ----------------------------------------------------------------------------- hard hash
+// Classic RACE with hard P-bit hashes (hard_kernels.cuh): scratch layout and launches.
+struct HardPlan {
+  int G;
+  int64_t seg_len;
+  size_t off_qid, off_kid, off_cseg, off_cinit, off_vseg, off_vinit, off_num, off_cnt, bytes;
+};
+
+HardPlan hard_plan(const race_args_t* a) {
+  HardPlan p;
+  const int R = 1 << a->P;
+  const int64_t chunks = (a->N + hard::kHC - 1) / hard::kHC;
+  const int64_t units = (int64_t)a->H * a->L;
+  int64_t G = std::max<int64_t>(1, (2 * kPlanSMs + units - 1) / units);
+  G = std::min<int64_t>(G, chunks);
+  p.seg_len = ((chunks + G - 1) / G) * hard::kHC;
+  p.G = (int)((a->N + p.seg_len - 1) / p.seg_len);
+  const size_t rows = (size_t)a->H * a->N;
+  const size_t cells = (size_t)a->H * a->L * p.G * R;
+  size_t o = 0;
+  p.off_qid = o;   o = align_up(o + rows * a->L);
+  p.off_kid = o;   o = align_up(o + rows * a->L);
+  p.off_cseg = o;  o = align_up(o + cells * sizeof(int));
+  p.off_cinit = o; o = align_up(o + cells * sizeof(int));
+  p.off_vseg = o;  o = align_up(o + cells * kD * sizeof(float));
+  p.off_vinit = o; o = align_up(o + cells * kD * sizeof(float));
+  p.off_num = o;   o = align_up(o + rows * kD * sizeof(float));
+  p.off_cnt = o;   o = align_up(o + rows * sizeof(int));
+  p.bytes = o;
+  return p;
+}
+
+template <typename T>
+race_status_t hard_ids(const race_args_t* a, const T* x, const float* W, uint8_t* ids,
+                       cudaStream_t s) {
+  const int64_t w_hs = a->w_per_head ? (int64_t)a->L * kD * a->P : 0;
+  RACE_LAUNCH("hard_ids", s);
+  hard::k_hard_ids<T><<<dim3((unsigned)((a->N + 31) / 32), a->H), hard::kHT, 0, s>>>(
+      x, W, ids, a->N, a->L, a->P, w_hs);
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
+template <typename T, typename TO>
+race_status_t hard_forward(const race_args_t* a, const T* q, const T* k, const T* v,
+                           const float* W, TO* out, int* counts, char* ws, cudaStream_t s) {
+  const HardPlan p = hard_plan(a);
+  const int R = 1 << a->P;
+  auto* qid = reinterpret_cast<uint8_t*>(ws + p.off_qid);
+  auto* kid = reinterpret_cast<uint8_t*>(ws + p.off_kid);
+  int* cseg = reinterpret_cast<int*>(ws + p.off_cseg);
+  int* cinit = reinterpret_cast<int*>(ws + p.off_cinit);
+  float* vseg = reinterpret_cast<float*>(ws + p.off_vseg);
+  float* vinit = reinterpret_cast<float*>(ws + p.off_vinit);
+  float* num = reinterpret_cast<float*>(ws + p.off_num);
+  int* cnt = counts ? counts : reinterpret_cast<int*>(ws + p.off_cnt);
+  const size_t rows = (size_t)a->H * a->N;
+  race_status_t st = hard_ids<T>(a, q, W, qid, s);
+  if (st != RACE_OK) return st;
+  st = hard_ids<T>(a, k, W, kid, s);
+  if (st != RACE_OK) return st;
+  RACE_CU(cudaMemsetAsync(num, 0, rows * kD * sizeof(float), s));
+  RACE_CU(cudaMemsetAsync(cnt, 0, rows * sizeof(int), s));
+  const dim3 grid(p.G, a->L, a->H);
+  int have_init = 0;
+  if (!a->causal || p.G > 1) {
+    RACE_CU(set_smem(hard::k_hard_seg<T>, hard::seg_smem(R)));
+    {
+      RACE_LAUNCH("hard_segments", s);
+      hard::k_hard_seg<T><<<grid, hard::kHT, hard::seg_smem(R), s>>>(kid, v, cseg, vseg, a->N,
+                                                                    a->L, R, p.G, p.seg_len);
+    }
+    RACE_CU(cudaGetLastError());
+    {
+      RACE_LAUNCH("hard_scan", s);
+      hard::k_hard_scan<<<dim3((R * kDV + 255) / 256, a->H * a->L), 256, 0, s>>>(
+          cseg, vseg, cinit, vinit, R, p.G, a->causal ? 0 : 2);
+    }
+    RACE_CU(cudaGetLastError());
+    have_init = 1;
+  }
+  RACE_CU(set_smem(hard::k_hard_sweep<T>, hard::sweep_smem(R)));
+  {
+    RACE_LAUNCH("hard_sweep", s);
+    hard::k_hard_sweep<T><<<grid, hard::kHT, hard::sweep_smem(R), s>>>(
+        qid, kid, v, cinit, vinit, num, cnt, a->N, a->L, R, p.G, p.seg_len, a->causal,
+        have_init);
+  }
+  RACE_CU(cudaGetLastError());
+  {
+    RACE_LAUNCH("hard_normalize", s);
+    hard::k_hard_normalize<TO><<<(unsigned)((rows * kD + 255) / 256), 256, 0, s>>>(
+        num, cnt, out, (int64_t)rows);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
+}
+
 // Scratch: the caller's, or stream-ordered memory of our own.
 struct Scratch {
   char* ptr = nullptr;
@@ -1050,6 +1149,53 @@ race_status_t race_forward_stream(const void* q, const void* k, const void* v,
   cy.out = state_out;
   cy.on = true;
   return forward_impl(q, k, v, W, out, a, reinterpret_cast<cudaStream_t>(stream), &cy);
+}
+
+race_status_t race_hard_workspace_size(const race_args_t* a, size_t* bytes) {
+  if (bytes) *bytes = 0;
+  if (!bytes) return RACE_ERR_INVALID_ARG;
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  *bytes = hard_plan(a).bytes;
+  return RACE_OK;
+}
+
+race_status_t race_hard_forward(const void* q, const void* k, const void* v, const float* W,
+                                void* out, int* counts, const race_args_t* a,
+                                race_stream_t stream) {
+  NvtxRange r("race_hard_forward");
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  const void* ptrs[] = {q, k, v, W, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return RACE_ERR_INVALID_ARG;
+  if (counts && !aligned16(counts)) return RACE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Scratch sc;
+  st = sc.acquire(a, hard_plan(a).bytes, s);
+  if (st != RACE_OK) return st;
+#define RACE_HARD(T, TO)                                                                    \
+  return hard_forward<T, TO>(a, static_cast<const T*>(q), static_cast<const T*>(k),       \
+                             static_cast<const T*>(v), W, static_cast<TO*>(out), counts,  \
+                             sc.ptr, s)
+  if (a->dtype == RACE_BF16) {
+    if (a->out_dtype == RACE_BF16) RACE_HARD(__nv_bfloat16, __nv_bfloat16);
+    RACE_HARD(__nv_bfloat16, float);
+  }
+  if (a->out_dtype == RACE_BF16) RACE_HARD(float, __nv_bfloat16);
+  RACE_HARD(float, float);
+#undef RACE_HARD
+}
+
+race_status_t race_hard_hash(const void* x, const float* W, uint8_t* ids, const race_args_t* a,
+                             race_stream_t stream) {
+  race_status_t st = check_args(a);
+  if (st != RACE_OK) return st;
+  if (!x || !W || !ids || !aligned16(x) || !aligned16(W)) return RACE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (a->dtype == RACE_BF16)
+    return hard_ids<__nv_bfloat16>(a, static_cast<const __nv_bfloat16*>(x), W, ids, s);
+  return hard_ids<float>(a, static_cast<const float*>(x), W, ids, s);
 }
 
 race_status_t race_workspace_size(const race_args_t* a, int backward, size_t* bytes) {

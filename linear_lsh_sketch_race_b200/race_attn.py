@@ -33,7 +33,8 @@ EXPORTED = ("race_args_init", "race_forward", "race_backward", "race_forward_ex"
             "race_backward_ex", "race_workspace_size", "race_hash", "race_device_status",
             "race_status_string", "race_version", "race_timing_enable",
             "race_timing_report", "race_launch_count", "race_forward_noalloc",
-            "race_selftest_wait_timeout", "race_forward_stream")
+            "race_selftest_wait_timeout", "race_forward_stream", "race_hard_forward",
+            "race_hard_workspace_size", "race_hard_hash")
 
 
 class RaceArgs(ctypes.Structure):
@@ -85,6 +86,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.race_backward_ex.argtypes = [vp] * 10 + [pargs, vp]
     lib.race_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, pargs, vp]
     lib.race_forward_stream.argtypes = [vp, vp, vp, vp, vp, vp, vp, pargs, vp]
+    lib.race_hard_forward.argtypes = [vp, vp, vp, vp, vp, vp, pargs, vp]
+    lib.race_hard_workspace_size.argtypes = [pargs, ctypes.POINTER(ctypes.c_size_t)]
+    lib.race_hard_hash.argtypes = [vp, vp, vp, pargs, vp]
     lib.race_workspace_size.argtypes = [pargs, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.race_hash.argtypes = [vp, vp, vp, pargs, vp]
     lib.race_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -101,7 +105,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("race_forward", "race_backward", "race_forward_ex", "race_backward_ex",
                  "race_forward_noalloc", "race_workspace_size", "race_hash", "race_device_status",
                  "race_timing_enable", "race_timing_report", "race_selftest_wait_timeout",
-                 "race_forward_stream"):
+                 "race_forward_stream", "race_hard_forward", "race_hard_workspace_size",
+                 "race_hard_hash"):
         getattr(lib, name).restype = i32
     lib.race_version.restype = i32
     _lib = lib
@@ -295,6 +300,42 @@ def backward(q, k, v, W, tau, causal, out, dout, den=None, chunk=0, impl="auto",
     a = make_args(q, W, tau, causal, out.dtype, chunk, impl, den, workspace, gdt)
     race_backward_ex(q, k, v, W, out, dout, dq, dk, dv, dW, a, stream)
     return dq, dk, dv, dW
+
+
+def race_hard_forward(q, k, v, W, out, counts, args: RaceArgs, stream=None):
+    _check(load().race_hard_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out),
+                                    _ptr(counts), ctypes.byref(args), _stream(stream)),
+           "race_hard_forward")
+
+
+def race_hard_workspace_size(args: RaceArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().race_hard_workspace_size(ctypes.byref(args), ctypes.byref(n)),
+           "race_hard_workspace_size")
+    return n.value
+
+
+def race_hard_hash(x, W, ids, args: RaceArgs, stream=None):
+    _check(load().race_hard_hash(_ptr(x), _ptr(W), _ptr(ids), ctypes.byref(args),
+                                 _stream(stream)), "race_hard_hash")
+
+
+def hard_forward(q, k, v, W, causal, out_dtype=None, stream=None):
+    """Classic RACE with hard hashes: returns (out, counts) with counts int32 [H, N]."""
+    out_dtype = out_dtype or q.dtype
+    out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    counts = torch.empty(q.shape[:2], dtype=torch.int32, device=q.device)
+    a = make_args(q, W, 1.0, causal, out_dtype)
+    race_hard_forward(q, k, v, W, out, counts, a, stream)
+    return out, counts
+
+
+def hard_hash(x, W, stream=None):
+    """Bucket ids uint8 [H, N, L] of the hard hash."""
+    H, N, _ = x.shape
+    ids = torch.empty((H, N, W.shape[-3]), dtype=torch.uint8, device=x.device)
+    race_hard_hash(x, W, ids, make_args(x, W, 1.0, False), stream)
+    return ids
 
 
 def state_shape(H: int, L: int, P: int):

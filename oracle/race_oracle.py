@@ -111,6 +111,38 @@ def hard_hash(x: np.ndarray, W: np.ndarray) -> np.ndarray:
     return np.sum(bits << np.arange(W.shape[2])[None, None, :], axis=-1)
 
 
+def hard_forward(q, k, v, W, causal):
+    """The classic RACE estimator with hard hashes (the tau -> 0 limit of the soft one)
+    for one head: count arrays of bucket collisions ([JA] §2.1: repeated arrays of count
+    estimators, bucket aggregation; [KO] §2: L tables of P-bit buckets).
+
+    A_ij = number of tables l with h_l(q_i) == h_l(k_j), over the attended set J(i);
+    o_i = sum_j A_ij v_j / sum_j A_ij, and o_i = 0 where no key collides with q_i in any
+    table (reading: the ratio is undefined there; the soft estimator never has this case).
+    Returns (o [N, d], den [N] integer collision counts)."""
+    v = np.asarray(v, dtype=np.float64)
+    hq, hk = hard_hash(q, W), hard_hash(k, W)              # [N, L]
+    A = (hq[:, None, :] == hk[None, :, :]).sum(axis=2).astype(np.float64)
+    A = A * _mask(len(q), causal)
+    den = A.sum(axis=1)
+    num = A @ v
+    o = np.where(den[:, None] > 0, num / np.maximum(den, 1.0)[:, None], 0.0)
+    return o, den.astype(np.int64)
+
+
+def hard_counts(x, v, W):
+    """Count arrays of one head: C[l, b] = number of keys in bucket b of table l and
+    S[l, b] = sum of their values ([JA] §2.1 bucket aggregation with hard hashes)."""
+    h = hard_hash(x, W)
+    L, R = W.shape[0], 1 << W.shape[2]
+    C = np.zeros((L, R), dtype=np.int64)
+    S = np.zeros((L, R, v.shape[1]))
+    for l in range(L):
+        np.add.at(C[l], h[:, l], 1)
+        np.add.at(S[l], h[:, l], np.asarray(v, dtype=np.float64))
+    return C, S
+
+
 def angular_kernel(q: np.ndarray, k: np.ndarray, P: int) -> np.ndarray:
     """sim[i, j] = (1 - arccos(qhat_i . khat_j)/pi)^P  ([JA] §2.1, sim equation)."""
     c = np.clip(normalize(q) @ normalize(k).T, -1.0, 1.0)

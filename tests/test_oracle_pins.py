@@ -424,3 +424,55 @@ def test_multihead_wrappers():
         assert np.allclose(o[h], oh) and np.allclose(den[h], dh)
         tot += oracle.backward(q[h], k[h], v[h], W, 0.5, True, g[h])[3]
     assert np.allclose(dW, tot)
+
+
+# --------------------------------------------------------------------------- #
+# hard-hash RACE (classic count arrays)
+# --------------------------------------------------------------------------- #
+def test_hard_forward_matches_scalar_loops():
+    """A second route with explicit loops over tables and keys on a small case."""
+    rng = np.random.default_rng(40)
+    N, d, L, P = 23, 5, 3, 2
+    q, k, v, W = _rand_case(rng, N, d, L, P)
+    for causal in (False, True):
+        o, den = oracle.hard_forward(q, k, v, W, causal)
+        hq, hk = oracle.hard_hash(q, W), oracle.hard_hash(k, W)
+        for i in range(N):
+            cnt, acc = 0, np.zeros(d)
+            for j in range(N):
+                if causal and j > i:
+                    continue
+                m = sum(int(hq[i, l] == hk[j, l]) for l in range(L))
+                cnt += m
+                acc += m * v[j]
+            assert den[i] == cnt
+            assert np.allclose(o[i], acc / cnt if cnt else 0.0, rtol=1e-13, atol=1e-14)
+
+
+def test_hard_forward_is_the_soft_estimator_as_tau_goes_to_zero():
+    """With tau -> 0 every soft assignment is one-hot at the hard bucket, so the soft
+    weights phi(q).phi(k) become (number of colliding tables) / L."""
+    rng = np.random.default_rng(41)
+    q, k, v, W = _rand_case(rng, 40, 8, 4, 3)
+    o_h, den_h = oracle.hard_forward(q, k, v, W, True)
+    with np.errstate(invalid="ignore"):   # rows with no collision: 0/0 in the soft form
+        o_s, den_s = oracle.direct_forward(q, k, v, W, 1e-6, True)
+    ok = den_h > 0
+    assert ok.sum() > 30
+    assert np.allclose(den_s[ok] * 4, den_h[ok], rtol=1e-6, atol=1e-6)
+    assert np.allclose(o_s[ok], o_h[ok], rtol=1e-6, atol=1e-6)
+
+
+def test_hard_counts_are_histograms_and_give_the_noncausal_estimator():
+    rng = np.random.default_rng(42)
+    q, k, v, W = _rand_case(rng, 200, 8, 5, 4)
+    C, S = oracle.hard_counts(k, v, W)
+    assert (C.sum(axis=1) == 200).all()
+    assert np.allclose(S.sum(axis=1), np.tile(v.sum(axis=0), (5, 1)))
+    hq = oracle.hard_hash(q, W)
+    num = sum(S[l, hq[:, l]] for l in range(5))
+    den = sum(C[l, hq[:, l]] for l in range(5))
+    o, den2 = oracle.hard_forward(q, k, v, W, False)
+    assert (den == den2).all()
+    nz = den > 0
+    assert np.allclose(num[nz] / den[nz, None], o[nz], rtol=1e-12)
