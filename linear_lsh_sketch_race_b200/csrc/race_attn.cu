@@ -584,12 +584,13 @@ BwPlan make_bw_plan(const race_args_t* a) {
   const int LP = a->L * a->P;
   p.lps = (LP + 7) / 8 * 8;   // 16-byte rows of bf16 per-plane gradients
   p.w_hs = a->w_per_head ? (int64_t)LP * kD : 0;
-  // finalize blocks per head: about one CTA per SM over all heads (tensor-core finalize,
-  // 128-token tiles) or four (CUDA-core finalize, 64-token tiles)
+  // finalize blocks per head: at most one CTA per SM over all heads (tensor-core finalize,
+  // 128-token tiles, one resident CTA per SM) or four (CUDA-core finalize, 64-token tiles),
+  // rounded down so that the grid is a single wave
   {
     const int tile = LP <= tc::kFzMaxLP ? 128 : tc::kFinTok;
     const int64_t per_sm = LP <= tc::kFzMaxLP ? 1 : 4;
-    const int64_t want = (per_sm * kPlanSMs + a->H - 1) / a->H;
+    const int64_t want = std::max<int64_t>(1, per_sm * kPlanSMs / a->H);
     b.fin_blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (a->N + tile - 1) / tile));
   }
   const size_t st = (size_t)a->H * p.n_rg * p.G * 256 * tc::kNV * sizeof(float);
