@@ -20,6 +20,7 @@
 #include "tc_sweep_pipe.cuh"
 #include "tc_backward.cuh"
 #include "tc_finalize.cuh"
+#include "tc_bwd_pipe.cuh"
 #include "hard_kernels.cuh"
 
 namespace race {
@@ -553,11 +554,16 @@ bool tc_backward_supported(const race_args_t* a) {
   return LR % 256 == 0 && (int64_t)a->L * a->P <= tc::kMaxLP;
 }
 
+// The causal sweeps at R = 256 run as the pipelined kernel k_bwd_pipe (two CTAs per table).
+bool bw_pipelined(const race_args_t* a) { return a->P == 8 && a->causal; }
+
 struct BwPlan {
   tc::Params prm;
   int fin_blocks;
+  bool pipe;                 // k_bwd_pipe for the q and k sweeps
+  int64_t inv_stride;        // row stride of the 1/|x| scratch (whole chunks)
   size_t off_fwd, off_rinv, off_gdot, off_rq, off_rk, off_rg, off_rr, off_duq, off_duk,
-      off_seg, off_init, off_part, bytes;
+      off_seg, off_init, off_part, off_inv, off_z, off_gext, bytes;
 };
 
 BwPlan make_bw_plan(const race_args_t* a) {
@@ -571,7 +577,9 @@ BwPlan make_bw_plan(const race_args_t* a) {
   p.tables = 256 / p.R;
   p.np = ((p.tables * a->P + 15) / 16) * 16;
   p.n_rg = (a->L * p.R) / 256;
-  const int64_t units = (int64_t)a->H * p.n_rg;
+  b.pipe = bw_pipelined(a);
+  // CTAs per (head, segment): one per row group, two per table for the pipelined sweep
+  const int64_t units = (int64_t)a->H * p.n_rg * (b.pipe ? 2 : 1);
   const int64_t tiles = (a->N + tc::kC - 1) / tc::kC;
   int64_t G = a->causal ? std::max<int64_t>(1, kPlanSMs / units)
                         : std::max<int64_t>(1, (kPlanSMs + units - 1) / units);
@@ -612,6 +620,16 @@ BwPlan make_bw_plan(const race_args_t* a) {
   b.off_seg = o;  o = align_up(o + st);
   b.off_init = o; o = align_up(o + st);
   b.off_part = o; o = align_up(o + 2 * (size_t)a->H * b.fin_blocks * LP * kD * sizeof(float));
+  // 1/|x| of q and k rows, [2][H][inv_stride], and their scaled projections,
+  // [2][H][L][inv_stride][8] (pipelined sweep only)
+  b.inv_stride = tiles * tc::kC;
+  b.off_inv = o;
+  if (b.pipe) o = align_up(o + 2 * (size_t)a->H * b.inv_stride * sizeof(float));
+  b.off_z = o;
+  if (b.pipe) o = align_up(o + 2 * (size_t)a->H * a->L * b.inv_stride * 8 * sizeof(float));
+  // extra feature columns of g', [H][N][16] bf16 (pipelined sweep only)
+  b.off_gext = o;
+  if (b.pipe) o = align_up(o + (size_t)rows * 16 * sizeof(__nv_bfloat16));
   b.bytes = o;
   return b;
 }
@@ -653,6 +671,30 @@ race_status_t bw_dispatch(int P, int mode, bool rev, const tc::Params& prm,
     case 8: return bw_launch<8>(mode, rev, prm, xa, xb, fa, fb, ea, eb, ra, rb, W, init, seg, du, name, s);
   }
   return RACE_ERR_UNSUPPORTED;
+}
+
+// The pipelined causal sweep at R = 256: grid (G, 2 * tables, H) in clusters of the two
+// halves of a table.
+race_status_t bw_pipe_launch(bool rev, const tc::Params& prm, const CUtensorMap& fa,
+                             const CUtensorMap& fb, const CUtensorMap& ge, const float* rinv,
+                             const float* za, const float* zb, const float* inv_a,
+                             int64_t zstride, const float* init, __nv_bfloat16* du,
+                             const char* name, cudaStream_t s) {
+  const dim3 grid(prm.G, 2 * prm.n_rg, prm.H);
+  const size_t smem = tc::BPSmem::alloc;
+  if (rev) {
+    RACE_CU(set_smem(tc::k_bwd_pipe<true>, smem));
+    RACE_LAUNCH(name, s);
+    tc::k_bwd_pipe<true><<<grid, tc::kBPThreads, smem, s>>>(fa, fb, ge, rinv, za, zb, inv_a,
+                                                             zstride, init, du, prm);
+  } else {
+    RACE_CU(set_smem(tc::k_bwd_pipe<false>, smem));
+    RACE_LAUNCH(name, s);
+    tc::k_bwd_pipe<false><<<grid, tc::kBPThreads, smem, s>>>(fa, fb, ge, rinv, za, zb, inv_a,
+                                                              zstride, init, du, prm);
+  }
+  RACE_CU(cudaGetLastError());
+  return RACE_OK;
 }
 
 template <int MT, typename TG>
@@ -738,6 +780,33 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
     return RACE_ERR_CUDA;
   const int mode = a->causal ? tc::kSweep : tc::kReadout;
   const int RD = 256 * tc::kNV;
+  float* inv_q = reinterpret_cast<float*>(ws + pl.off_inv);
+  float* inv_k = inv_q + (size_t)a->H * pl.inv_stride;
+  float* z_q = reinterpret_cast<float*>(ws + pl.off_z);
+  float* z_k = z_q + (size_t)a->H * a->L * pl.inv_stride * 8;
+  auto* gext = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_gext);
+  CUtensorMap tge;
+  if (pl.pipe) {
+    {
+      const size_t zsm = tc::zproj_smem(a->L);
+      const int per_sm = 512 / tc::zproj_cols(a->L);
+      const int64_t tiles = (a->N + tc::kC - 1) / tc::kC;
+      const int64_t want = std::max<int64_t>(1, (int64_t)kPlanSMs * per_sm / (2 * a->H));
+      const unsigned gx = (unsigned)std::min<int64_t>(tiles, want);
+      RACE_CU(set_smem(tc::k_bwd_zproj, zsm));
+      RACE_LAUNCH("tc_bwd_zproj", s);
+      tc::k_bwd_zproj<<<dim3(gx, a->H, 2), tc::kZpThreads, zsm, s>>>(
+          xq, xk, W, pl.prm.w_hs, z_q, inv_q, a->N, a->H, a->L, pl.inv_stride,
+          pl.prm.two_over_tau);
+    }
+    RACE_CU(cudaGetLastError());
+    {
+      RACE_LAUNCH("tc_bwd_gext", s);
+      tc::k_bwd_gext<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(gdot, gext, rows);
+    }
+    RACE_CU(cudaGetLastError());
+    if (!tc::encode_gext_tmap(&tge, gext, a->N, a->H)) return RACE_ERR_CUDA;
+  }
   // ---- q side: dP(q) = r (g' S^T + mask(g' [v|1]^T) p(k)), S over keys j <= i
   tc::Params prm = pl.prm;
   if (!a->causal || prm.G > 1) {
@@ -752,8 +821,10 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
     RACE_CU(cudaGetLastError());
     prm.have_init = 1;
   }
-  st = bw_dispatch(a->P, mode, false, prm, xq, xk, fg, fv, gdot, nullptr, rinv, nullptr, W,
-                   init, seg, duq, "tc_bwd_q", s);
+  st = pl.pipe ? bw_pipe_launch(false, prm, fg, fv, tge, rinv, z_q, z_k, inv_q,
+                                pl.inv_stride, init, duq, "tc_bwd_q", s)
+               : bw_dispatch(a->P, mode, false, prm, xq, xk, fg, fv, gdot, nullptr, rinv,
+                             nullptr, W, init, seg, duq, "tc_bwd_q", s);
   if (st != RACE_OK) return st;
   // ---- k side: dP(k) = [v|1] T^T + mask([v|1] g'^T) (r p(q)), T over queries i >= j
   prm = pl.prm;
@@ -769,8 +840,10 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
     RACE_CU(cudaGetLastError());
     prm.have_init = 1;
   }
-  st = bw_dispatch(a->P, mode, a->causal != 0, prm, xk, xq, fv, fg, nullptr, gdot, nullptr,
-                   rinv, W, init, seg, duk, "tc_bwd_k", s);
+  st = pl.pipe ? bw_pipe_launch(true, prm, fv, fg, tge, rinv, z_k, z_q, inv_k,
+                                pl.inv_stride, init, duk, "tc_bwd_k", s)
+               : bw_dispatch(a->P, mode, a->causal != 0, prm, xk, xq, fv, fg, nullptr, gdot,
+                             nullptr, rinv, W, init, seg, duk, "tc_bwd_k", s);
   if (st != RACE_OK) return st;
   // ---- dv_j = sum_{i >= j} w_ij r_i g_i: the forward sweep with queries k, keys q (each
   //      p(q_i) scaled by r_i) and values g (sequence reversed for the causal case)

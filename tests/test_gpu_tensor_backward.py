@@ -112,10 +112,12 @@ def test_tensor_backward_near_one_hot_assignments():
     assert max(errs.values()) <= TOL_BWD, errs
 
 
-def test_tensor_backward_ragged_chunk_edges():
-    # lengths at and around the 128-token chunk, several segments of unequal length
+@pytest.mark.parametrize("P", [7, 8])
+def test_tensor_backward_ragged_chunk_edges(P):
+    # lengths at and around the 128-token chunk, several segments of unequal length (at
+    # P = 8 the causal sweeps run as the two-CTA pipelined kernel)
     for N in (127, 128, 129, 640, 1537):
-        wl, x, g = _case(N, 1, 2, 7, 0.5, True, seed=N)
+        wl, x, g = _case(N, 1, 2, P, 0.5, True, seed=N)
         grads, _ = _run(wl, x, g)
         errs = _errors(grads, _refs(wl, x), N)
         assert max(errs.values()) <= TOL_BWD, (N, errs)
