@@ -14,15 +14,16 @@
 // come from a tensor-core pre-pass (k_bwd_zproj), one 4 KB bulk copy per side and step.
 //
 // Per step i (128 tokens of side a and of side b):
-//   warp 16 (issuer A): XY(i) = X Y^T (-> DW); UPD(i): S += p(b)^T Y; dP(i) = X S^T (state
-//                       hi + lo) + mask(XY) p(b) into one of two dP buffers
+//   warp 16 (issuer A): UPD(i): S += p(b)^T Y; dP(i) = X S^T (state hi + lo) + mask(XY) p(b)
+//                       into one of two dP buffers; XY(i+1) = X Y^T (-> DW)
 //   warp 17 (issuer B): the copies of features and projections
 //   warps 0-3   (EXP):  p(b) of step i into one of two tiles
-//   warps 4-7   (MASK): mask(XY(i)) rounded to bf16 in place (the A operand of dP)
+//   warps 4-7, 12-15 (MASK + STAGE, one 64-key block and part of the state per warp):
+//                       after dP(i-1), S_{i-1} from tensor memory into its bf16 hi + lo
+//                       copy for dP(i); mask(XY(i)) rounded to bf16 in place (the A
+//                       operand of dP(i))
 //   warps 8-11  (HASH): side-a logistic factors; reads dP(i), per-plane sums over the half
 //                       table, exchange, du' store
-//   warps 12-15 (STAGE): after dP(i), S_i from tensor memory into its bf16 hi + lo copy
-//                       for dP(i+1)
 // Every producer/consumer pair has its own mbarrier, every wait is bounded, and no
 // barrier can complete a phase twice ahead of one of its waiters (two-slot resources
 // have one barrier per slot).
@@ -39,7 +40,7 @@ constexpr int kBPThreads = 576;
 
 enum BPBar : int {
   bp_FA0 = 0, bp_FA1, bp_FB0, bp_FB1, bp_Z0, bp_Z1, bp_ZREAD0, bp_ZREAD1, bp_PB0, bp_PB1,
-  bp_PBU0, bp_PBU1, bp_PBD0, bp_PBD1, bp_XY0, bp_XY1, bp_INTRA, bp_DP0, bp_DP1,
+  bp_PBU0, bp_PBU1, bp_PBD0, bp_PBD1, bp_XY0, bp_XY1, bp_INTRA0, bp_INTRA1, bp_DP0, bp_DP1,
   bp_DPFREE0, bp_DPFREE1, bp_SBF, bp_XFULL, bp_XFREE, bp_COUNT
 };
 
@@ -150,14 +151,17 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < bp_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == bp_PB0 || i == bp_PB1 || i == bp_INTRA || i == bp_DPFREE0 || i == bp_DPFREE1 ||
-          i == bp_SBF)
-        cnt = 4;
+      if (i == bp_PB0 || i == bp_PB1 || i == bp_DPFREE0 || i == bp_DPFREE1) cnt = 4;
       if (i == bp_ZREAD0 || i == bp_ZREAD1) cnt = 8;   // EXP and HASH warps
-      if (i == bp_XFULL || i == bp_XFREE) cnt = 128;   // one arrival per thread of the peer
+      if (i == bp_INTRA0 || i == bp_INTRA1 || i == bp_SBF) cnt = 8;   // MASK + STAGE warps
+      if (i == bp_XFREE) cnt = 128;                    // one arrival per thread of the peer
       mbar_init(bar + i, cnt);
     }
     fence_mbar_init();
+    // the lower half expects the upper half's 128 x 32 bytes of step 0 (asynchronous
+    // stores completing on XFULL); each later step's expectation is posted after the
+    // previous step's exchange
+    if (hb == 0) mbar_arrive_expect_tx(bar + bp_XFULL, 128 * 32);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -264,19 +268,18 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
     };
     if (warp == 16) {
       // ---------------------------------------------------------- issuer A: XY, UPD, dP
-      // In tensor-core order per step: XY(i), then UPD(i) while the MASK warps round
-      // XY(i), then dP(i).
-      for (int i = 0; i < n && ok; ++i) {
-        if (lane == 0) BW_TRACE(i, 0);
+      // Tensor-core order: ... UPD(i), dP(i), XY(i+1), UPD(i+1), dP(i+1) ...  MMAs issued
+      // by one thread execute in issue order, so XY(i+1) overwrites DW only after dP(i)
+      // has read it, and runs while the STAGE warps copy S_i; the MASK warps round XY(i+1)
+      // while UPD(i+1) runs.
+      auto xy = [&](int i) {
         const int st = i & 1;
         const uint32_t fa = sb + (st ? BPSmem::fa1 : BPSmem::fa0);
         const uint32_t fb = sb + (st ? BPSmem::fb1 : BPSmem::fb0);
-        const uint32_t pbt = sb + (st ? BPSmem::pb1 : BPSmem::pb0);
-        // DW and the X slot of step i-1 are free once dP(i-1) completed
-        if (i > 0 && !wait(bp_DP0 + ((i - 1) & 1), (uint32_t)((i - 1) >> 1) & 1)) break;
-        if (lane == 0) BW_TRACE(i, 1);
-        if (!wait(bp_FA0 + st, (uint32_t)(i >> 1) & 1) || !wait(bp_FB0 + st, (uint32_t)(i >> 1) & 1))
-          break;
+        if (lane == 0) BW_TRACE(i, 27);
+        if (!wait(bp_FA0 + st, (uint32_t)(i >> 1) & 1)) return false;
+        if (lane == 0) BW_TRACE(i, 28);
+        if (!wait(bp_FB0 + st, (uint32_t)(i >> 1) & 1)) return false;
         if (lane == 0) BW_TRACE(i, 2);
         tc_fence_after();
         if (elect_one()) {
@@ -285,10 +288,18 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
             umma_ss(tmem + BPTm::DW, sdesc(fa + s * 4096, 16, 256, kSwizzle32B),
                     sdesc(fb + s * 4096, 16, 256, kSwizzle32B), id_128, s > 0);
           umma_commit(bar + bp_XY0 + st);
-          if (i > 0 && i + 1 < n) load_fa(i + 1);
         }
         __syncwarp();
-        // state update with p(b) of step i (after S_{i-1} was copied out)
+        return true;
+      };
+      if (n > 0) xy(0);
+      for (int i = 0; i < n && ok; ++i) {
+        if (lane == 0) BW_TRACE(i, 0);
+        const int st = i & 1;
+        const uint32_t fa = sb + (st ? BPSmem::fa1 : BPSmem::fa0);
+        const uint32_t fb = sb + (st ? BPSmem::fb1 : BPSmem::fb0);
+        const uint32_t pbt = sb + (st ? BPSmem::pb1 : BPSmem::pb0);
+        // state update with p(b) of step i, after S_{i-1} was copied out
         if (!wait(bp_PB0 + st, (uint32_t)(i >> 1) & 1)) break;
         if (i > 0 && !wait(bp_SBF, (uint32_t)(i - 1) & 1)) break;
         if (lane == 0) BW_TRACE(i, 4);
@@ -302,7 +313,8 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
           umma_commit(bar + bp_PBU0 + st);
         }
         __syncwarp();
-        if (!wait(bp_INTRA, (uint32_t)i & 1)) break;
+        // dP(i) once XY(i) is rounded (and dP buffer st was read two steps ago)
+        if (!wait(bp_INTRA0 + st, (uint32_t)(i >> 1) & 1)) break;
         if (i > 1 && !wait(bp_DPFREE0 + st, (uint32_t)((i - 2) >> 1) & 1)) break;
         if (lane == 0) BW_TRACE(i, 3);
         tc_fence_after();
@@ -317,12 +329,20 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
           }
           const uint64_t dpb = sdesc(pbt, 16384, 1024, kSwizzle128B);
 #pragma unroll
-          for (int s = 0; s < 8; ++s)
-            umma_ts(dP, tmem + BPTm::DW + s * 8, dpb + 128 * s, id_d3, 1);
+          for (int s = 0; s < 8; ++s)   // keys 16 s ..: block s/4, packed columns 8 (s % 4)
+            umma_ts(dP, tmem + BPTm::DW + (s >> 2) * 64 + (s & 3) * 8, dpb + 128 * s, id_d3, 1);
           umma_commit(bar + bp_DP0 + st);
           umma_commit(bar + bp_PBD0 + st);
         }
         __syncwarp();
+        if (i + 1 < n && !xy(i + 1)) break;
+        // the X slot of step i is refilled with step i+2 once dP(i) has read it
+        if (i + 2 < n) {
+          if (!wait(bp_DP0 + st, (uint32_t)(i >> 1) & 1)) break;
+          if (lane == 0) BW_TRACE(i, 1);
+          if (elect_one()) load_fa(i + 2);
+          __syncwarp();
+        }
       }
     } else {
       // ---------------------------------------------------------- issuer B: copies
@@ -377,10 +397,12 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
       for (int p = 0; p < P; ++p) logistic_fast(z[p], sp[p], smv[p]);
       Corners k;
       corners_of(sp, smv, fb, k);
-      // p(b) tile slot free once UPD(i-2) and dP(i-2) have read it
+      // p(b) tile slot free once UPD(i-2) and dP(i-2) have read it; the expansion runs
+      // after MASK(i-1), alongside dP(i-1), off the CUDA-core work between dP(i-1) and dP(i)
       if (i > 1 && (!wait(bp_PBU0 + st, (uint32_t)((i - 2) >> 1) & 1) ||
                     !wait(bp_PBD0 + st, (uint32_t)((i - 2) >> 1) & 1)))
         break;
+      if (i > 0 && !wait(bp_INTRA0 + ((i - 1) & 1), (uint32_t)((i - 1) >> 1) & 1)) break;
       if (t == 0) BW_TRACE(i, 10);
       expand_half128(sb + (st ? BPSmem::pb1 : BPSmem::pb0), t, k, hb);
       fence_proxy_async();
@@ -388,58 +410,7 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
       if (lane == 0) mbar_arrive(bar + bp_PB0 + st);
       if (t == 0) BW_TRACE(i, 11);
     }
-  } else if (warp < 8) {
-    // ================================================================ MASK
-    const int q4 = warp - 4;
-    const int t = q4 * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    for (int i = 0; i < n; ++i) {
-      if (!wait(bp_XY0 + (i & 1), (uint32_t)(i >> 1) & 1)) break;
-      if (t == 0) BW_TRACE(i, 12);
-      tc_fence_after();
-      // key blocks in pairs: fp32 columns 64p .. 64p+63 -> bf16 pairs in 32p .. 32p+31,
-      // which the first pair has already read; packed in place in registers.  A pair that
-      // the mask keeps whole, or drops whole, for all 32 rows of this warp skips the
-      // comparisons, or the loads.
-#pragma unroll
-      for (int kp = 0; kp < 2; ++kp) {
-        const int j_lo = kp * 64, j_hi = kp * 64 + 63, t_lo = q4 * 32, t_hi = q4 * 32 + 31;
-        const bool all_kept = REV ? (j_lo >= t_hi) : (j_hi <= t_lo);
-        const bool all_dropped = REV ? (j_hi < t_lo) : (j_lo > t_hi);
-        uint32_t x[64];
-        if (all_dropped) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = 0u;
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tmem_ld16(tmem + lane_off + BPTm::DW + kp * 64 + q * 16, x + q * 16);
-          tmem_ld_wait();
-          if (all_kept) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              x[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int j0 = kp * 64 + 2 * e;
-              const bool k0 = REV ? (j0 >= t) : (j0 <= t);
-              const bool k1 = REV ? (j0 + 1 >= t) : (j0 + 1 <= t);
-              x[e] = pack_bf16(k0 ? __uint_as_float(x[2 * e]) : 0.f,
-                               k1 ? __uint_as_float(x[2 * e + 1]) : 0.f);
-            }
-          }
-        }
-        tmem_st16(tmem + lane_off + BPTm::DW + kp * 32, x);
-        tmem_st16(tmem + lane_off + BPTm::DW + kp * 32 + 16, x + 16);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar + bp_INTRA);
-      if (t == 0) BW_TRACE(i, 13);
-    }
-  } else if (warp < 12) {
+  } else if (warp >= 8 && warp < 12) {
     // ================================================================ HASH (side a)
     const int q4 = warp - 8;
     const int t = q4 * 32 + lane;
@@ -453,6 +424,7 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
       const bool valid = row < s1;
       const float fa = fa_next;   // row factor (0 past the end), loaded a step ahead
       if (i + 1 < n) fa_next = row_factor(A_IS_G, i + 1, t);
+      if (t == 0) BW_TRACE(i, 26);
       // projections and logistic factors of side a
       if (!wait(bp_Z0 + st, (uint32_t)(i >> 1) & 1)) break;
       if (t == 0) BW_TRACE(i, 15);
@@ -462,7 +434,9 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
       const float inv = valid ? reinterpret_cast<const float*>(sm + BPSmem::inva + st * 512)[t] : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar + bp_ZREAD0 + st);
-      float sp[P], lo[8], hi[16];
+      // corner factors: low corners e (planes 0-2), and the high corner c = 4 q + g of the
+      // half as p34[g] (planes 3-4) times p567[q] (planes 5-6 and plane 7 = hb)
+      float sp[P], lo[8], p34[4], p567[4];
       {
         float sm_[P];
 #pragma unroll
@@ -470,40 +444,72 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
 #pragma unroll
         for (int b = 0; b < 8; ++b)
           lo[b] = ((b & 1) ? sp[0] : sm_[0]) * ((b & 2) ? sp[1] : sm_[1]) * ((b & 4) ? sp[2] : sm_[2]);
-        hi[0] = hb ? sp[7] : sm_[7];
-        kron_tree<3, 7>(hi, sp, sm_);              // planes 3-6 over the 16 high corners
+        const float f7 = hb ? sp[7] : sm_[7];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          p34[g] = ((g & 1) ? sp[3] : sm_[3]) * ((g & 2) ? sp[4] : sm_[4]);
+          p567[g] = ((g & 1) ? sp[5] : sm_[5]) * ((g & 2) ? sp[6] : sm_[6]) * f7;
+        }
       }
-      // per-plane sums over this half's 128 corners
+      // per-plane sums over this half's 128 corners, after MASK(i+1): alongside dP(i+1),
+      // off the CUDA-core work between dP(i) and dP(i+1)
       if (!wait(bp_DP0 + st, (uint32_t)(i >> 1) & 1)) break;
+      if (i + 1 < n && !wait(bp_INTRA0 + ((i + 1) & 1), (uint32_t)((i + 1) >> 1) & 1)) break;
       if (t == 0) BW_TRACE(i, 16);
       tc_fence_after();
-      float Ts = 0.f, As[P];
-#pragma unroll
-      for (int p = 0; p < P; ++p) As[p] = 0.f;
+      // Packed pairs over the 8 low corners e of each group of 8 rows: with
+      // m_e = lo_e dP_e, S1 = (m0+m2, m1+m3), S2 = (m4+m6, m5+m7), T = S1 + S2 and
+      // U = (m2+m6, m3+m7): sum_e m_e = T.x + T.y, plane 0 = T.y, plane 1 = U.x + U.y,
+      // plane 2 = S2.x + S2.y; planes 3-6 take hi_c T where bit p-3 of the group c is set.
+      uint64_t accT = 0, accU = 0, accS2 = 0, acc3 = 0, acc4 = 0, acc5 = 0, acc6 = 0;
+      const uint64_t lo01 = pair_f32x2(lo[0], lo[1]), lo23 = pair_f32x2(lo[2], lo[3]);
+      const uint64_t lo45 = pair_f32x2(lo[4], lo[5]), lo67 = pair_f32x2(lo[6], lo[7]);
       const uint32_t dpc = tmem + lane_off + (st ? BPTm::DP1 : BPTm::DP0);
+      // 16 columns per piece; the load of piece q+1 is in flight while piece q is summed
+      uint32_t xb[2][16];
+      tmem_ld16(dpc, xb[0]);
+      tmem_ld_wait();
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        uint32_t x[32];
-        tmem_ld16(dpc + qq * 32, x);
-        tmem_ld16(dpc + qq * 32 + 16, x + 16);
-        tmem_ld_wait();
+      for (int qq = 0; qq < 8; ++qq) {
+        if (qq + 1 < 8) tmem_ld16(dpc + (qq + 1) * 16, xb[(qq + 1) & 1]);
+        const uint32_t* x = xb[qq & 1];
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-          const int c = qq * 4 + g8;                  // high corner index (planes 3-6)
-          float m[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) m[e] = lo[e] * __uint_as_float(x[g8 * 8 + e]);
-          const float zz = ((m[0] + m[1]) + (m[2] + m[3])) + ((m[4] + m[5]) + (m[6] + m[7]));
-          const float hz = hi[c];
-          Ts = fmaf(hz, zz, Ts);
-          As[0] = fmaf(hz, (m[1] + m[3]) + (m[5] + m[7]), As[0]);
-          As[1] = fmaf(hz, (m[2] + m[3]) + (m[6] + m[7]), As[1]);
-          As[2] = fmaf(hz, (m[4] + m[5]) + (m[6] + m[7]), As[2]);
-          const float w = hz * zz;
-#pragma unroll
-          for (int p = 3; p < 7; ++p)
-            if ((c >> (p - 3)) & 1) As[p] += w;
+        for (int g8 = 0; g8 < 2; ++g8) {
+          const int c = qq * 2 + g8;                  // high corner index (planes 3-6)
+          const uint32_t* xg = x + g8 * 8;
+          const uint64_t m01 = mul_f32x2(lo01, pair_u32x2(xg[0], xg[1]));
+          const uint64_t m23 = mul_f32x2(lo23, pair_u32x2(xg[2], xg[3]));
+          const uint64_t m45 = mul_f32x2(lo45, pair_u32x2(xg[4], xg[5]));
+          const uint64_t m67 = mul_f32x2(lo67, pair_u32x2(xg[6], xg[7]));
+          const uint64_t s2 = add_f32x2(m45, m67);
+          const uint64_t tt = add_f32x2(add_f32x2(m01, m23), s2);
+          const uint64_t uu = add_f32x2(m23, m67);
+          const uint64_t hz = bcast_f32x2(p34[c & 3] * p567[c >> 2]);
+          const uint64_t ht = mul_f32x2(hz, tt);
+          accT = add_f32x2(accT, ht);
+          accU = fma_f32x2(hz, uu, accU);
+          accS2 = fma_f32x2(hz, s2, accS2);
+          if (c & 1) acc3 = add_f32x2(acc3, ht);
+          if (c & 2) acc4 = add_f32x2(acc4, ht);
+          if (c & 4) acc5 = add_f32x2(acc5, ht);
+          if (c & 8) acc6 = add_f32x2(acc6, ht);
         }
+        if (qq + 1 < 8) tmem_ld_wait();
+      }
+      float Ts, As[P];
+      {
+        const float2 vt = unpack_f32x2(accT), vu = unpack_f32x2(accU), vs = unpack_f32x2(accS2);
+        const float2 v3 = unpack_f32x2(acc3), v4 = unpack_f32x2(acc4);
+        const float2 v5 = unpack_f32x2(acc5), v6 = unpack_f32x2(acc6);
+        Ts = vt.x + vt.y;
+        As[0] = vt.y;
+        As[1] = vu.x + vu.y;
+        As[2] = vs.x + vs.y;
+        As[3] = v3.x + v3.y;
+        As[4] = v4.x + v4.y;
+        As[5] = v5.x + v5.y;
+        As[6] = v6.x + v6.y;
+        As[7] = 0.f;
       }
       tc_fence_before();
       __syncwarp();
@@ -515,25 +521,32 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
 #pragma unroll
       for (int p = 0; p < P; ++p) d[p] = sc * (As[p] - sp[p] * Ts);
       // ---- the two halves' sums meet in the lower half (one exchange slot)
+      if (t == 0) BW_TRACE(i, 18);
       if (hb) {
         if (i > 0 && !mbar_wait_cluster(bar + bp_XFREE, (uint32_t)(i - 1) & 1)) { ok = false; }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint32_t dst = map_to_rank(xch, peer);
-        st_cluster_v4(dst, d[0], d[1], d[2], d[3]);
-        st_cluster_v4(dst + 16, d[4], d[5], d[6], d[7]);
-        mbar_arrive_remote(map_to_rank(smem_u32(bar + bp_XFULL), peer));
+        const uint32_t rbar = map_to_rank(smem_u32(bar + bp_XFULL), peer);
+        st_async_v4(dst, d[0], d[1], d[2], d[3], rbar);
+        st_async_v4(dst + 16, d[4], d[5], d[6], d[7], rbar);
       } else {
         if (!mbar_wait_cluster(bar + bp_XFULL, (uint32_t)i & 1)) { ok = false; }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (t == 0) BW_TRACE(i, 19);
+        // the next step's data cannot arrive before this thread's XFREE arrival below
+        if (t == 0 && i + 1 < n) mbar_arrive_expect_tx(bar + bp_XFULL, 128 * 32);
         float o[8];
         ld_shared_v4f(xch, o);
         ld_shared_v4f(xch + 16, o + 4);
-        mbar_arrive_remote(map_to_rank(smem_u32(bar + bp_XFREE), peer));
 #pragma unroll
         for (int p = 0; p < P; ++p) d[p] += o[p];
+        // the slot's values are in registers (used above): the peer may refill it
+        asm volatile("" ::"f"(d[0]), "f"(d[1]), "f"(d[2]), "f"(d[3]), "f"(d[4]), "f"(d[5]),
+                     "f"(d[6]), "f"(d[7]));
+        mbar_arrive_remote_relaxed(map_to_rank(smem_u32(bar + bp_XFREE), peer));
+        if (t == 0) BW_TRACE(i, 20);
         if (valid) {
           const size_t off = ((size_t)h * prm.N + row) * prm.lps + (size_t)l * P;
           uint32_t hp[4], lp[4];
@@ -547,38 +560,85 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
           *reinterpret_cast<uint4*>(du_out + (size_t)prm.H * prm.N * prm.lps + off) =
               make_uint4(lp[0], lp[1], lp[2], lp[3]);
         }
+        if (t == 0) BW_TRACE(i, 25);
       }
     }
   } else {
-    // ================================================================ STAGE: state copy
-    // After dP(i) (whose commit also covers UPD(i), issued before it by the same thread):
-    // S_i from tensor memory, 16 columns at a time, into the bf16 hi + lo copy read by
-    // dP(i+1); UPD(i+1) waits for this read.
-    const int q4 = warp - 12;
+    // ================================================================ MASK + STAGE
+    // Warps 4-7 and 12-15: lane quarter q4 = warp % 4, key block kb = warp / 12 (keys
+    // 64 kb .. 64 kb + 63; state columns 40 kb .. 40 kb + 39).  Per step i: STAGE(i-1) after
+    // dP(i-1), which also covers UPD(i-1) issued before it by the same thread: S_{i-1}
+    // from tensor memory into its bf16 hi + lo copy read by dP(i); then MASK(i): the
+    // key block of XY(i), masked and rounded to bf16 pairs in place, in the first 32
+    // columns of the block (the A operand of dP(i)).
+    const int q4 = warp & 3, kb = warp >= 12 ? 1 : 0;
     const int t = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const int m0 = kb * 5;                         // state columns 8 m0 .. 8 m0 + 39
+    const int j_lo = kb * 64, j_hi = kb * 64 + 63, t_lo = q4 * 32, t_hi = q4 * 32 + 31;
+    const bool all_kept = REV ? (j_lo >= t_hi) : (j_hi <= t_lo);
+    const bool all_dropped = REV ? (j_hi < t_lo) : (j_lo > t_hi);
     for (int i = 0; i < n; ++i) {
-      if (!wait(bp_DP0 + (i & 1), (uint32_t)(i >> 1) & 1)) break;
-      if (t == 0) BW_TRACE(i, 23);
-      tc_fence_after();
+      if (i > 0) {
+        if (!wait(bp_DP0 + ((i - 1) & 1), (uint32_t)((i - 1) >> 1) & 1)) break;
+        if (t == 0) BW_TRACE(i - 1, 23);
+        tc_fence_after();
+        // this warp's 40 state columns (8-column groups m0 .. m0+4) in one round of loads
+        uint32_t r[40];
 #pragma unroll
-      for (int b = 0; b < 5; ++b) {
-        uint32_t r[16], hi[8], lo[8];
-        tmem_ld16(tmem + lane_off + BPTm::S + b * 16, r);
+        for (int j = 0; j < 5; ++j) tmem_ld8(tmem + lane_off + BPTm::S + (m0 + j) * 8, r + 8 * j);
         tmem_ld_wait();
-        split_state8(r, hi, lo);
-        split_state8(r + 8, hi + 4, lo + 4);
-        const uint32_t o0 = state_sw32_off(t, 2 * b), o1 = state_sw32_off(t, 2 * b + 1);
-        st_shared_v4(sb + BPSmem::shi + o0, hi[0], hi[1], hi[2], hi[3]);
-        st_shared_v4(sb + BPSmem::slo + o0, lo[0], lo[1], lo[2], lo[3]);
-        st_shared_v4(sb + BPSmem::shi + o1, hi[4], hi[5], hi[6], hi[7]);
-        st_shared_v4(sb + BPSmem::slo + o1, lo[4], lo[5], lo[6], lo[7]);
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+          uint32_t hi[4], lo[4];
+          split_state8(r + 8 * j, hi, lo);
+          const uint32_t o = state_sw32_off(t, m0 + j);
+          st_shared_v4(sb + BPSmem::shi + o, hi[0], hi[1], hi[2], hi[3]);
+          st_shared_v4(sb + BPSmem::slo + o, lo[0], lo[1], lo[2], lo[3]);
+        }
+        tc_fence_before();
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + bp_SBF);
+        if (t == 0) BW_TRACE(i - 1, 24);
       }
+      if (!wait(bp_XY0 + (i & 1), (uint32_t)(i >> 1) & 1)) break;
+      if (t == 0) BW_TRACE(i, 12);
+      tc_fence_after();
+      // two halves of 32 keys: fp32 columns 64 kb + 32 h .. -> bf16 pairs in 64 kb + 16 h ..,
+      // which this warp has already read
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t x[32];
+        if (all_dropped) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) x[e] = 0u;
+        } else {
+          tmem_ld16(tmem + lane_off + BPTm::DW + kb * 64 + hh * 32, x);
+          tmem_ld16(tmem + lane_off + BPTm::DW + kb * 64 + hh * 32 + 16, x + 16);
+          tmem_ld_wait();
+          if (all_kept) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              x[e] = pack_bf16(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int j0 = kb * 64 + hh * 32 + 2 * e;
+              const bool k0 = REV ? (j0 >= t) : (j0 <= t);
+              const bool k1 = REV ? (j0 + 1 >= t) : (j0 + 1 <= t);
+              x[e] = pack_bf16(k0 ? __uint_as_float(x[2 * e]) : 0.f,
+                               k1 ? __uint_as_float(x[2 * e + 1]) : 0.f);
+            }
+          }
+        }
+        tmem_st16(tmem + lane_off + BPTm::DW + kb * 64 + hh * 16, x);
+      }
+      tmem_st_wait();
       tc_fence_before();
-      fence_proxy_async();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar + bp_SBF);
-      if (t == 0) BW_TRACE(i, 24);
+      if (lane == 0) mbar_arrive(bar + bp_INTRA0 + (i & 1));
+      if (t == 0) BW_TRACE(i, 13);
     }
   }
   tc_fence_before();
