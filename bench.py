@@ -400,35 +400,90 @@ def run_ours(args, wl: I.Workload):
 
 def run_e2e(args, wl, x, a, ra, dev, stream, world, backward):
     """Same step through the public API with host inputs: pinned host -> device copies
-    of q, k, v (and dO), the step, device -> host copies of the results."""
+    of q, k, v (and dO), the step, device -> host copies of the results.
+
+    The heads go in two groups (when the head count is even): the inputs of group 2
+    upload while group 1 computes, and the results of group 1 download while group 2
+    computes, on two copy streams (one cudaMemcpyAsync per tensor slice).  With 4 of 8
+    heads per call the sweeps still fill one wave of CTAs, so the grouping costs the
+    kernels nothing; dW of the shared planes is the sum of the groups' dW."""
     try:
         import torch.distributed as dist
         names = ["q", "k", "v"] + (["dout"] if backward else [])
+        H = x["q"].shape[0]
+        ng = 2 if H % 2 == 0 and H >= 2 else 1
+        hg = H // ng
         host = {n: torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True) for n in names}
         for n in names:
             host[n].copy_(x[n])
         dev_in = {n: torch.empty_like(x[n]) for n in names}
         W = x["W"]
         out = torch.empty_like(x["q"])
-        outs = [out]
+        den = torch.empty(x["q"].shape[:2], dtype=torch.float32, device=dev)
+        per_head = [out]
         if backward:
-            grads = [torch.empty_like(x["q"]), torch.empty_like(x["k"]),
-                     torch.empty_like(x["v"]), torch.empty_like(W)]
-            outs += grads
-        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+            dq, dk, dv = (torch.empty_like(x[n]) for n in ("q", "k", "v"))
+            per_head += [dq, dk, dv]
+            dWg = [torch.empty_like(W) for _ in range(ng)]
+            dW = torch.empty_like(W)
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in per_head]
+        host_dW = torch.empty(W.shape, dtype=W.dtype, pin_memory=True) if backward else None
         h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-        d2h = sum(t.numel() * t.element_size() for t in outs)
+        d2h = sum(t.numel() * t.element_size() for t in per_head)
+        if backward:
+            d2h += W.numel() * W.element_size()
+        sl = [slice(g * hg, (g + 1) * hg) for g in range(ng)]
+        ga = []
+        for g in range(ng):
+            ag = ra.make_args(x["q"][sl[g]], W, wl.tau, wl.causal, chunk=wl.chunk,
+                              impl=args.kernels, den=den[sl[g]])
+            ag.workspace, ag.workspace_bytes = a.workspace, a.workspace_bytes
+            ga.append(ag)
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        state = {"computed": [None] * ng, "downloaded": [None] * ng}
 
         def step():
-            for n in names:
-                dev_in[n].copy_(host[n], non_blocking=True)
-            ra.race_forward_ex(dev_in["q"], dev_in["k"], dev_in["v"], W, out, a, stream)
+            uploaded = []
+            for g in range(ng):
+                with torch.cuda.stream(up):
+                    if state["computed"][g] is not None:   # last step's compute read them
+                        up.wait_event(state["computed"][g])
+                    for n in names:
+                        dev_in[n][sl[g]].copy_(host[n][sl[g]], non_blocking=True)
+                    e = ev()
+                    e.record(up)
+                    uploaded.append(e)
+            for g in range(ng):
+                stream.wait_event(uploaded[g])
+                if state["downloaded"][g] is not None:   # last step's results were read
+                    stream.wait_event(state["downloaded"][g])
+                d = {n: dev_in[n][sl[g]] for n in names}
+                ra.race_forward_ex(d["q"], d["k"], d["v"], W, out[sl[g]], ga[g], stream)
+                if backward:
+                    ra.race_backward_ex(d["q"], d["k"], d["v"], W, out[sl[g]], d["dout"],
+                                        dq[sl[g]], dk[sl[g]], dv[sl[g]], dWg[g], ga[g], stream)
+                e = ev()
+                e.record(stream)
+                state["computed"][g] = e
+                with torch.cuda.stream(down):
+                    down.wait_event(e)
+                    for t, hst in zip(per_head, host_out):
+                        hst[sl[g]].copy_(t[sl[g]], non_blocking=True)
+                    e2 = ev()
+                    e2.record(down)
+                    state["downloaded"][g] = e2
             if backward:
-                ra.race_backward_ex(dev_in["q"], dev_in["k"], dev_in["v"], W, out,
-                                    dev_in["dout"], *grads, a, stream)
-                allreduce_dw(grads[3], world)
-            for t, h in zip(outs, host_out):
-                h.copy_(t, non_blocking=True)
+                torch.sum(torch.stack(dWg), dim=0, out=dW)
+                allreduce_dw(dW, world)
+                e = ev()
+                e.record(stream)
+                with torch.cuda.stream(down):
+                    down.wait_event(e)
+                    host_dW.copy_(dW, non_blocking=True)
+            end = ev()
+            end.record(down)
+            stream.wait_event(end)
 
         n = max(1, min(args.steps, args.e2e_steps))
         step()
@@ -446,7 +501,7 @@ def run_e2e(args, wl, x, a, ra, dev, stream, world, backward):
         tokens = wl.batch * wl.N * world
         return {"value": tokens / (ms / 1000), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": ms, "steps": n}
+                "ms_per_step": ms, "steps": n, "head_groups": ng}
     except Exception as e:  # pinned host memory can be short on some hosts
         return {"value": None, "unit": "tokens/s", "error": repr(e)[:200]}
 
