@@ -38,7 +38,7 @@ def test_traffic_scales_with_token_heads_and_only_for_the_captured_configuration
     assert bench.kernel_traffic("tc_causal_sweep", WL.replace(N=131072, H=8)) == \
         pytest.approx(946.05e6)
     assert bench.kernel_traffic("tc_bwd_q", WL.replace(N=131072, H=8)) == \
-        pytest.approx(1319.13e6)
+        pytest.approx(1475.26e6 + 563.68e6)
     assert bench.kernel_traffic("tc_causal_sweep", WL.replace(P=6)) is None
     assert bench.kernel_traffic("tc_bwd_finalize", WL) is None
 
@@ -49,12 +49,19 @@ def _profile_mb(name):
     return float(m.group(1).replace(",", "")) + float(m.group(2).replace(",", ""))
 
 
+def _pipe_profile_mb(side):
+    """DRAM read + write (MB) of one instantiation in the pipelined backward's summary."""
+    text = open(os.path.join(ROOT, "profiles", "tc_bwd_pipe__causal_h8_n131072_L16_P8.md")).read()
+    m = re.search(r"`k_bwd_pipe<%d>`[^|]*\|[^|]*\| ([\d,.]+) MB \| ([\d,.]+) MB" % side, text)
+    return float(m.group(1).replace(",", "")) + float(m.group(2).replace(",", ""))
+
+
 def test_traffic_constants_match_the_committed_capture_summaries():
     sweep = _profile_mb("tc_causal_sweep__causal_h8_n131072_L16_P8.md")
-    bwd = _profile_mb("tc_bwd_phi__causal_h8_n131072_L16_P8.md")
     small = WL.replace(N=131072, H=8)
     assert bench.kernel_traffic("tc_causal_sweep", small) / 1e6 == pytest.approx(sweep, abs=1)
-    assert bench.kernel_traffic("tc_bwd_q", small) / 1e6 == pytest.approx(bwd, abs=1)
+    assert bench.kernel_traffic("tc_bwd_q", small) / 1e6 == pytest.approx(_pipe_profile_mb(0), abs=1)
+    assert bench.kernel_traffic("tc_bwd_k", small) / 1e6 == pytest.approx(_pipe_profile_mb(1), abs=1)
 
 
 def test_roofline_takes_the_dominant_kernel_and_keeps_the_forward_sweep():
