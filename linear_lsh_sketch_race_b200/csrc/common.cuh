@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bounds.h"
 #include "race_attn.h"
 
 namespace race {
@@ -35,6 +36,21 @@ __device__ __forceinline__ void raise_status(uint32_t bits) {
 }
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// RACE_IN_RANGE(i, n): in the bounds-checked build (-DRACE_BOUNDS_CHECK) false, with the
+// bounds bit of the device status flag raised, when i is outside [0, n); the caller then
+// skips the access (no trap, no early return, so no barrier is left waiting).  In the
+// normal build the condition is the constant true and costs nothing.
+#ifdef RACE_BOUNDS_CHECK
+__device__ __forceinline__ bool checked_index(int64_t i, int64_t n) {
+  if (index_in_range(i, n)) return true;
+  raise_status(kStatusBounds);
+  return false;
+}
+#define RACE_IN_RANGE(i, n) (::race::checked_index((int64_t)(i), (int64_t)(n)))
+#else
+#define RACE_IN_RANGE(i, n) true
+#endif
 
 // ---------------------------------------------------------------- element access
 template <typename T>

@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kHT) k_hard_seg(const uint8_t* __restrict__ ki
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t j = s0 + warp; j < s1; j += kHT / 32) {   // one warp per key
     const int b = kid[((size_t)h * N + j) * L + l];
+    if (!RACE_IN_RANGE(b, R)) continue;   // bounds-checked build: a corrupt id is skipped
     const T* vj = v + ((size_t)h * N + j) * kD;
     atomicAdd(&V[b * kD + lane], to_f(vj[lane]));
     atomicAdd(&V[b * kD + lane + 32], to_f(vj[lane + 32]));
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(kHT) k_hard_sweep(
     for (int t = warp; t < nt; t += kHT / 32) {
       const int64_t i = c0 + t;
       const int b = qid[((size_t)h * N + i) * L + l];
+      if (!RACE_IN_RANGE(b, R)) continue;
       float a0 = V[b * kD + lane], a1 = V[b * kD + lane + 32];
       int n = C[b];
       if (causal) {
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kHT) k_hard_sweep(
       __syncthreads();
       for (int t = warp; t < nt; t += kHT / 32) {
         const int b = kb[t];
+        if (!RACE_IN_RANGE(b, R)) continue;
         atomicAdd(&V[b * kD + lane], vc[t * kD + lane]);
         atomicAdd(&V[b * kD + lane + 32], vc[t * kD + lane + 32]);
         if (lane == 0) atomicAdd(&C[b], 1);

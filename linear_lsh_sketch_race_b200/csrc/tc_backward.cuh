@@ -578,10 +578,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           else hash_bwd_half<P, 1>(dp, lo, hi, Ts, As);
         }
         if (s_abort) break;
-        if (valid) {
+        const size_t off = ((size_t)h * prm.N + t0 + t) * prm.lps + (size_t)l0 * P;
+        if (valid && RACE_IN_RANGE(off + TABLES * P - 1, (int64_t)prm.H * prm.N * prm.lps)) {
           // du' = du / max(|x|, eps) as a bf16 hi + lo pair (about 16 significant bits):
           // the finalize then multiplies by W and by the unnormalised x tile directly
-          const size_t off = ((size_t)h * prm.N + t0 + t) * prm.lps + (size_t)l0 * P;
           __nv_bfloat16* dh = du_out + off;
           __nv_bfloat16* dl = du_out + (size_t)prm.H * prm.N * prm.lps + off;
           const float sc = prm.two_over_tau * fa * inv_a;

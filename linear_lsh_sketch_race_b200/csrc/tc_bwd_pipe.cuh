@@ -547,8 +547,8 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
                      "f"(d[6]), "f"(d[7]));
         mbar_arrive_remote_relaxed(map_to_rank(smem_u32(bar + bp_XFREE), peer));
         if (t == 0) BW_TRACE(i, 20);
-        if (valid) {
-          const size_t off = ((size_t)h * prm.N + row) * prm.lps + (size_t)l * P;
+        const size_t off = ((size_t)h * prm.N + row) * prm.lps + (size_t)l * P;
+        if (valid && RACE_IN_RANGE(off + P - 1, (int64_t)prm.H * prm.N * prm.lps)) {
           uint32_t hp[4], lp[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
