@@ -21,6 +21,7 @@
 #include "tc_backward.cuh"
 #include "tc_finalize.cuh"
 #include "tc_bwd_pipe.cuh"
+#include "tc_build_pipe.cuh"
 #include "hard_kernels.cuh"
 
 namespace race {
@@ -458,7 +459,14 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
     tc::k_sweep<P, TABLES><<<grid, tc::kSwThreads, tc::SwSmem::alloc, s>>>(tq, tk, tv, W, init,
                                                                           num, kscale, prm);
   } else if (mode == tc::kSweep) RACE_TC(tc::kSweep, "tc_causal_sweep_rows128");
-  else if (mode == tc::kBuild) RACE_TC(tc::kBuild, "tc_sketch_build");
+  else if (mode == tc::kBuild && P < 8 && prm.rows == 256 && !prm.have_init) {
+    if constexpr (P < 8) {
+      RACE_CU(set_smem(tc::k_build_pipe<P>, tc::BldSmem::alloc));
+      RACE_LAUNCH("tc_sketch_build", s);
+      tc::k_build_pipe<P><<<grid, tc::kBPipeThreads, tc::BldSmem::alloc, s>>>(tk, tv, W, seg,
+                                                                             kscale, prm);
+    }
+  } else if (mode == tc::kBuild) RACE_TC(tc::kBuild, "tc_sketch_build");
   else RACE_TC(tc::kReadout, "tc_readout");
 #undef RACE_TC
   RACE_CU(cudaGetLastError());
