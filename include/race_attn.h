@@ -38,6 +38,16 @@
  * (cudaStream_t; NULL is the legacy default stream).  They never print, abort or
  * exit.  Argument errors are reported before anything is enqueued.
  *
+ * Threads and state.  The compute calls keep no host state between calls: several
+ * host threads may call them at once, each with its own workspace (race_args_t
+ * .workspace, or the library's own allocation).  State shared by the whole process:
+ * the device status flag (one word per device, raised by any call on it and read and
+ * cleared by race_device_status), the static scratch of race_forward_noalloc (see
+ * there), the launch counter (atomic), the profiling registry of race_timing_* (a
+ * mutex guards it; while recording is on every launch of every thread adds events to
+ * it), and two values fixed at the first call: the driver entry point used to build
+ * TMA descriptors and the RACE_NVTX switch.
+ *
  * Supported sizes: d = 64; 1 <= P <= 8; L >= 1 with L * 2^P <= 16384; N >= 1;
  * H >= 1; tau finite and > 0.  Other d values give RACE_ERR_UNSUPPORTED.
  */
