@@ -22,6 +22,7 @@
 #include "tc_finalize.cuh"
 #include "tc_bwd_pipe.cuh"
 #include "tc_build_pipe.cuh"
+#include "tc_readout_pipe.cuh"
 #include "hard_kernels.cuh"
 
 namespace race {
@@ -467,7 +468,14 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
                                                                              kscale, prm);
     }
   } else if (mode == tc::kBuild) RACE_TC(tc::kBuild, "tc_sketch_build");
-  else RACE_TC(tc::kReadout, "tc_readout");
+  else if (P < 8 && prm.rows == 256 && prm.have_init) {
+    if constexpr (P < 8) {
+      RACE_CU(set_smem(tc::k_readout_pipe<P>, tc::RdSmem::alloc));
+      RACE_LAUNCH("tc_readout", s);
+      tc::k_readout_pipe<P><<<grid, tc::kRPipeThreads, tc::RdSmem::alloc, s>>>(tq, W, init,
+                                                                              num, prm);
+    }
+  } else RACE_TC(tc::kReadout, "tc_readout");
 #undef RACE_TC
   RACE_CU(cudaGetLastError());
   return RACE_OK;
