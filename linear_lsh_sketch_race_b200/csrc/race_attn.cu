@@ -785,7 +785,8 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   }
   {
     RACE_LAUNCH("tc_bwd_prep", s);
-    tc::k_bwd_prep<__nv_bfloat16, TO><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+    const int64_t blocks = std::min<int64_t>((rows + 31) / 32, (int64_t)kPlanSMs * 16);
+    tc::k_bwd_prep<__nv_bfloat16, TO><<<(unsigned)blocks, 256, 0, s>>>(
         dout, out, num, a->den, gdot, rinv, rows, (float)a->L);
   }
   RACE_CU(cudaGetLastError());
@@ -887,7 +888,7 @@ race_status_t tc_backward(const race_args_t* a, const __nv_bfloat16* q, const __
   if (st != RACE_OK) return st;
   {
     RACE_LAUNCH("tc_bwd_dv_out", s);
-    tc::k_dv_out<TG><<<(unsigned)((rows * kD + 255) / 256), 256, 0, s>>>(
+    tc::k_dv_out<TG><<<dim3((unsigned)((a->N + 15) / 16), a->H), 256, 0, s>>>(
         vnum, dv, a->N, a->H, a->causal);
   }
   RACE_CU(cudaGetLastError());

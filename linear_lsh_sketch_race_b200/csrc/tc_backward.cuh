@@ -658,16 +658,31 @@ __global__ void k_bwd_prep(const T* __restrict__ dout, const TO* __restrict__ ou
                            const float* __restrict__ num, const float* __restrict__ den_in,
                            float* __restrict__ gdot, float* __restrict__ rinv, int64_t rows,
                            float L) {
-  const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (i >= rows) return;
-  const float den = den_in ? den_in[i] * L : num[i * kNumStride + kD];
-  const float g0 = to_f(dout[i * kD + 2 * lane]), g1 = to_f(dout[i * kD + 2 * lane + 1]);
-  const float o0 = to_f(out[i * kD + 2 * lane]), o1 = to_f(out[i * kD + 2 * lane + 1]);
-  const float c = simt::warp_sum(g0 * o0 + g1 * o1);
-  if (lane == 0) {
-    gdot[i] = -c;
-    rinv[i] = 1.0f / den;
+  // eight lanes per row (8 elements each), four rows per warp per pass, grid-stride
+  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t i = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
+       i - (lane >> 3) < rows; i += warps * 4) {
+    const bool valid = i < rows;
+    float c = 0.f;
+    if (valid) {
+      float g[8], o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        g[e] = to_f(dout[i * kD + sub * 8 + e]);
+        o[e] = to_f(out[i * kD + sub * 8 + e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) c = fmaf(g[e], o[e], c);
+    }
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 4);
+    if (valid && sub == 0) {
+      const float den = den_in ? den_in[i] * L : num[i * kNumStride + kD];
+      gdot[i] = -c;
+      rinv[i] = 1.0f / den;
+    }
   }
 }
 
@@ -698,13 +713,18 @@ __global__ void k_reverse_rows(const __nv_bfloat16* __restrict__ src,
 template <typename T>
 __global__ void k_dv_out(const float* __restrict__ num, T* __restrict__ dv, int64_t N, int H,
                          int reversed) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (int64_t)H * N * kD) return;
-  const int64_t row = e / kD;
-  const int c = (int)(e % kD);
-  const int64_t h = row / N, n = row % N;
-  const int64_t src = reversed ? h * N + (N - 1 - n) : row;
-  dv[e] = from_f<T>(num[src * kNumStride + c]);
+  // grid (row blocks, H): sixteen threads per row, four columns (one float4) each
+  const int h = blockIdx.y;
+  const int64_t n = (int64_t)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4);
+  const int c4 = (threadIdx.x & 15) * 4;
+  if (n >= N) return;
+  const int64_t src = (int64_t)h * N + (reversed ? N - 1 - n : n);
+  const float4 v = *reinterpret_cast<const float4*>(num + src * kNumStride + c4);
+  T* d = dv + ((int64_t)h * N + n) * kD + c4;
+  d[0] = from_f<T>(v.x);
+  d[1] = from_f<T>(v.y);
+  d[2] = from_f<T>(v.z);
+  d[3] = from_f<T>(v.w);
 }
 
 // Hash backward, last steps, per token x (a row of q or k) on CUDA cores, for L * P above
