@@ -654,14 +654,15 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
 // Scaled projections of every row of q (side 0) and k (side 1) on every plane of every
 // table, z[side][h][l][n][p] = (x_n . W_l[:,p]) (2/tau) / max(|x_n|, eps) (float32, rows
 // padded to zstride, zero past N), and inv[side][h][n] = 1 / max(|x_n|, eps).
-// One 128-row tile per iteration: TMA x tile (128B swizzle) -> tcgen05 (A = x, B = W as a
-// bf16 hi + lo pair in the 16 columns of each table, N = 16 L in tiles of at most 256) ->
-// tensor memory -> 128 threads, one row each.  160 threads; warp 4 issues.
+// One 128-row tile per iteration: TMA x tile (128B swizzle, two slots: the next tile loads
+// while this one's epilogue runs) -> tcgen05 (A = x, B = W as a bf16 hi + lo pair in the
+// 16 columns of each table, N = 16 L in tiles of at most 256) -> tensor memory -> 128
+// threads, one row each, four tables per round of loads.  160 threads; warp 4 issues.
 constexpr int kZpThreads = 160;
 
 __host__ __device__ inline int zproj_cols(int L) { return 16 * L <= 256 ? 256 : 512; }
 inline size_t zproj_smem(int L) {
-  const size_t need = 16384 + (size_t)64 * 16 * L * 2 + 64 + 1024;
+  const size_t need = 2 * 16384 + (size_t)64 * 16 * L * 2 + 64 + 1024;
   // at most 512 / cols CTAs per SM, so that tensor-memory allocation never waits
   const size_t one_per_sm = 232448 / 2 + 1024;
   return zproj_cols(L) == 512 ? std::max(need, one_per_sm) : std::max(need, (size_t)232448 / 3 + 1024);
@@ -676,10 +677,11 @@ __global__ void __launch_bounds__(kZpThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  constexpr uint32_t kX = 0, kW = 16384;
+  constexpr uint32_t kX = 0, kW = 32768;                   // x: two 16 KB slots
   const int NC = 16 * L;                                   // B columns
   const uint32_t bars = kW + (uint32_t)64 * NC * 2;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + bars);  // 0: x tile, 1: MMA, 2: read
+  // 0, 1: x tile slots; 2: MMA done; 3: epilogue done reading (tensor memory, x slot)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + bars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + bars + 32);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, side = blockIdx.z;
@@ -688,7 +690,8 @@ __global__ void __launch_bounds__(kZpThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar + 0, 1);
     mbar_init(bar + 1, 1);
-    mbar_init(bar + 2, 4);
+    mbar_init(bar + 2, 1);
+    mbar_init(bar + 3, 4);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -713,60 +716,81 @@ __global__ void __launch_bounds__(kZpThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int64_t tiles = (N + kC - 1) / kC;
   const CUtensorMap* tx = side ? &tk : &tq;
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  const int its = first < tiles ? (int)((tiles - 1 - first) / step + 1) : 0;
   bool ok = true;
-  int it = 0;
-  for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++it) {
-    const uint32_t par = (uint32_t)it & 1;
-    if (warp == 4) {
+  if (warp == 4) {
+    auto load = [&](int it) {
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar + 0, 16384);
-        tma_load_3d(sm + kX, tx, 0, (int)(tile * kC), h, bar + 0);
+        mbar_arrive_expect_tx(bar + (it & 1), 16384);
+        tma_load_3d(sm + kX + (it & 1) * 16384, tx, 0, (int)((first + (int64_t)it * step) * kC),
+                    h, bar + (it & 1));
       }
       __syncwarp();
-      ok = mbar_wait(bar + 0, par);
+    };
+    if (its > 0) load(0);
+    for (int it = 0; it < its && ok; ++it) {
+      // the epilogue of tile it-1 has read the tensor memory and x slot (it+1) % 2
+      if (it >= 1) {
+        ok = mbar_wait(bar + 3, (uint32_t)(it - 1) & 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      if (it + 1 < its) load(it + 1);
+      ok = mbar_wait(bar + (it & 1), (uint32_t)(it >> 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       if (elect_one()) {
+        const uint32_t xs = sb + kX + (it & 1) * 16384;
         for (int nt = 0; nt < NC; nt += 256) {
           const int nw = NC - nt < 256 ? NC - nt : 256;
           const uint32_t id = idesc_bf16(128, nw, 0, 0);
 #pragma unroll
           for (int s = 0; s < 4; ++s)
-            umma_ss(tmem + nt, sdesc(sb + kX + s * 32, 16, 1024, kSwizzle128B),
+            umma_ss(tmem + nt, sdesc(xs + s * 32, 16, 1024, kSwizzle128B),
                     sdesc(sb + kW + nt * 128 + s * 256, 128, 1024, kSwizzleNone), id, s > 0);
         }
-        umma_commit(bar + 1);
+        umma_commit(bar + 2);
       }
       __syncwarp();
-      // the next tile's x copy overwrites the tile once the epilogue has read its norms
-      ok = mbar_wait(bar + 2, par);
-      ok = __all_sync(0xffffffffu, ok);
-    } else {
-      const int t = threadIdx.x;
-      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-      const int64_t row = tile * kC + t;
+    }
+  } else {
+    const int t = threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    for (int it = 0; it < its; ++it) {
+      const int64_t row = (first + (int64_t)it * step) * kC + t;
       // the x tile (TMA) for the norms, the projections (MMA) in tensor memory
-      if (!mbar_wait(bar + 0, par) || !mbar_wait(bar + 1, par)) ok = false;
+      if (!mbar_wait(bar + (it & 1), (uint32_t)(it >> 1) & 1) ||
+          !mbar_wait(bar + 2, (uint32_t)it & 1))
+        break;
       tc_fence_after();
-      const float iv = row_inv_norm(sm + kX, t);
+      const float iv = row_inv_norm(sm + kX + (it & 1) * 16384, t);
       const float sc = iv * two_over_tau;
-      for (int ll = 0; ll < L; ++ll) {
-        uint32_t r[16];
-        tmem_ld16(tmem + lane_off + ll * 16, r);
-        tmem_ld_wait();
-        float o[8];
+      for (int l4 = 0; l4 < L; l4 += 4) {   // four tables per round of loads
+        uint32_t r[4][16];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) o[p] = (__uint_as_float(r[p]) + __uint_as_float(r[8 + p])) * sc;
-        float4* dst = reinterpret_cast<float4*>(
-            z + ((((size_t)side * H + h) * L + ll) * zstride + row) * 8);
-        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+        for (int j = 0; j < 4; ++j)
+          if (l4 + j < L) tmem_ld16(tmem + lane_off + (l4 + j) * 16, r[j]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (l4 + j < L) {
+            float o[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p)
+              o[p] = (__uint_as_float(r[j][p]) + __uint_as_float(r[j][8 + p])) * sc;
+            float4* dst = reinterpret_cast<float4*>(
+                z + ((((size_t)side * H + h) * L + l4 + j) * zstride + row) * 8);
+            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+          }
+        }
       }
       inv[((size_t)side * H + h) * zstride + row] = iv;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar + 2);
+      if (lane == 0) mbar_arrive(bar + 3);
     }
   }
   tc_fence_before();
