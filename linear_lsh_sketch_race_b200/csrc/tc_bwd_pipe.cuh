@@ -14,8 +14,9 @@
 // come from a tensor-core pre-pass (k_bwd_zproj), one 4 KB bulk copy per side and step.
 //
 // Per step i (128 tokens of side a and of side b):
-//   warp 16 (issuer A): UPD(i): S += p(b)^T Y; dP(i) = X S^T (state hi + lo) + mask(XY) p(b)
-//                       into one of two dP buffers; XY(i+1) = X Y^T (-> DW)
+//   warp 16 (issuer A): dP(i) = X S^T (state hi + lo) + mask(XY) p(b) into one of two dP
+//                       buffers, with UPD(i): S += p(b)^T Y issued between the two parts
+//                       (the first needs no mask); XY(i+1) = X Y^T (-> DW)
 //   warp 17 (issuer B): the copies of features and projections
 //   warps 0-3   (EXP):  p(b) of step i into one of two tiles
 //   warps 4-7, 12-15 (MASK + STAGE, one 64-key block and part of the state per warp):
@@ -268,10 +269,9 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
     };
     if (warp == 16) {
       // ---------------------------------------------------------- issuer A: XY, UPD, dP
-      // Tensor-core order: ... UPD(i), dP(i), XY(i+1), UPD(i+1), dP(i+1) ...  MMAs issued
-      // by one thread execute in issue order, so XY(i+1) overwrites DW only after dP(i)
-      // has read it, and runs while the STAGE warps copy S_i; the MASK warps round XY(i+1)
-      // while UPD(i+1) runs.
+      // Tensor-core order: ... X S^T(i), UPD(i), intra(i), XY(i+1), X S^T(i+1), ...  MMAs
+      // issued by one thread execute in issue order, so XY(i+1) overwrites DW only after
+      // dP(i) has read it; X S^T(i+1) and UPD(i+1) run while XY(i+1) is masked.
       auto xy = [&](int i) {
         const int st = i & 1;
         const uint32_t fa = sb + (st ? BPSmem::fa1 : BPSmem::fa0);
@@ -299,24 +299,14 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
         const uint32_t fa = sb + (st ? BPSmem::fa1 : BPSmem::fa0);
         const uint32_t fb = sb + (st ? BPSmem::fb1 : BPSmem::fb0);
         const uint32_t pbt = sb + (st ? BPSmem::pb1 : BPSmem::pb0);
-        // state update with p(b) of step i, after S_{i-1} was copied out
+        // dP(i) in two parts: X S_{i-1}^T (hi + lo copy) as soon as the copy exists and
+        // dP buffer st was read two steps ago, then the state update, then the in-chunk
+        // term mask(XY(i)) p(b) once the MASK warps have rounded XY(i): the tensor core
+        // works on the first two while XY(i) is masked.
         if (!wait(bp_PB0 + st, (uint32_t)(i >> 1) & 1)) break;
         if (i > 0 && !wait(bp_SBF, (uint32_t)(i - 1) & 1)) break;
-        if (lane == 0) BW_TRACE(i, 4);
-        tc_fence_after();
-        if (elect_one()) {
-          const uint64_t dpb = sdesc(pbt, 16384, 1024, kSwizzle128B);
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            umma_ss(tmem + BPTm::S, dpb + 128 * s, sdesc(fb + s * 512, 4096, 256, kSwizzle32B),
-                    id_up, 1);
-          umma_commit(bar + bp_PBU0 + st);
-        }
-        __syncwarp();
-        // dP(i) once XY(i) is rounded (and dP buffer st was read two steps ago)
-        if (!wait(bp_INTRA0 + st, (uint32_t)(i >> 1) & 1)) break;
         if (i > 1 && !wait(bp_DPFREE0 + st, (uint32_t)((i - 2) >> 1) & 1)) break;
-        if (lane == 0) BW_TRACE(i, 3);
+        if (lane == 0) BW_TRACE(i, 4);
         tc_fence_after();
         if (elect_one()) {
           const uint32_t dP = tmem + (st ? BPTm::DP1 : BPTm::DP0);
@@ -327,6 +317,20 @@ __global__ void __launch_bounds__(kBPThreads, 1) __cluster_dims__(1, 2, 1)
                     s > 0);
             umma_ss(dP, xd, sdesc(sb + BPSmem::slo + s * 4096, 16, 256, kSwizzle32B), id_128, 1);
           }
+          // state update with p(b) of step i (S_{i-1} was copied out: SBF above)
+          const uint64_t dpb = sdesc(pbt, 16384, 1024, kSwizzle128B);
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            umma_ss(tmem + BPTm::S, dpb + 128 * s, sdesc(fb + s * 512, 4096, 256, kSwizzle32B),
+                    id_up, 1);
+          umma_commit(bar + bp_PBU0 + st);
+        }
+        __syncwarp();
+        if (!wait(bp_INTRA0 + st, (uint32_t)(i >> 1) & 1)) break;
+        if (lane == 0) BW_TRACE(i, 3);
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t dP = tmem + (st ? BPTm::DP1 : BPTm::DP0);
           const uint64_t dpb = sdesc(pbt, 16384, 1024, kSwizzle128B);
 #pragma unroll
           for (int s = 0; s < 8; ++s)   // keys 16 s ..: block s/4, packed columns 8 (s % 4)
