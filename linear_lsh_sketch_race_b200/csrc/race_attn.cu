@@ -449,10 +449,13 @@ race_status_t tc_launch(int mode, const tc::Params& prm, const CUtensorMap& tq,
   if (mode == tc::kSweep && P == 8 && prm.rows == 256 && inv_norms) {
     CUtensorMap tnum;
     if (!tc::encode_num_tmap(&tnum, num, prm.N, prm.H)) return RACE_ERR_CUDA;
-    RACE_CU(set_smem(tc::k_sweep_pipe, tc::SPSmem::alloc));
+    // A per-key factor means the backward's dv pass, which reads only the 64 value
+    // columns of num: the sweep then runs its value-side MMAs at N = 64 (no mass column).
+    auto* kern = kscale ? tc::k_sweep_pipe<64> : tc::k_sweep_pipe<80>;
+    RACE_CU(set_smem(kern, tc::SPSmem::alloc));
     RACE_LAUNCH("tc_causal_sweep", s);
-    tc::k_sweep_pipe<<<grid, tc::kSPThreads, tc::SPSmem::alloc, s>>>(
-        tq, tk, tv, W, init, inv_norms, inv_stride, tnum, num, kscale, prm);
+    kern<<<grid, tc::kSPThreads, tc::SPSmem::alloc, s>>>(tq, tk, tv, W, init, inv_norms,
+                                                        inv_stride, tnum, num, kscale, prm);
   } else if (mode == tc::kSweep && prm.rows == 256) {
     constexpr int TABLES = 256 >> P;
     RACE_CU(set_smem(tc::k_sweep<P, TABLES>, tc::SwSmem::alloc));

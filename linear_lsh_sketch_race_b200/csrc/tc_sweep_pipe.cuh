@@ -25,6 +25,11 @@
 // Every producer/consumer pair has its own mbarrier; a producer can be at most one
 // phase ahead of its consumer, so parity waits stay unambiguous.  An optional per-key
 // factor kscale[h][n] multiplies p(k_n) (the backward's dv pass uses the keys' 1/den').
+//
+// NVC is the width of the value side of every MMA: 80 = the 64 value columns and an atom
+// of ones whose first column accumulates the mass z (the forward, which needs the
+// denominator), or 64 = the values alone (the dv pass, which reads only the numerator;
+// its denominator column is written as zero).
 #pragma once
 
 #include "tc_sweep256.cuh"
@@ -68,10 +73,12 @@ struct SPTm {
 };
 
 
-// bf16 copy of the 80-column state row held in tensor-memory lane (this thread) at
-// column `col`: two batches of loads (48 + 32 columns), one wait each, packed to 40
-// bf16 pairs.  After this returns the tensor-memory row may be overwritten.
+// bf16 copy of the NVC-column state row held in tensor-memory lane (this thread) at
+// column `col`: two batches of loads (48 + NVC - 48 columns), one wait each, packed to
+// NVC / 2 bf16 pairs.  After this returns the tensor-memory row may be overwritten.
+template <int NVC>
 __device__ __forceinline__ void restage_load(uint32_t taddr, uint32_t* pk) {
+  static_assert(NVC == 64 || NVC == 80, "value width");
   uint32_t v[48];
   tmem_ld16(taddr, v);
   tmem_ld16(taddr + 16, v + 16);
@@ -79,20 +86,22 @@ __device__ __forceinline__ void restage_load(uint32_t taddr, uint32_t* pk) {
   tmem_ld_wait();
 #pragma unroll
   for (int e = 0; e < 24; ++e) pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-  tmem_ld16(taddr + 48, v);
-  tmem_ld16(taddr + 64, v + 16);
+#pragma unroll
+  for (int b = 0; b < (NVC - 48) / 16; ++b) tmem_ld16(taddr + 48 + 16 * b, v + 16 * b);
   tmem_ld_wait();
 #pragma unroll
-  for (int e = 0; e < 16; ++e)
+  for (int e = 0; e < (NVC - 48) / 2; ++e)
     pk[24 + e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
 }
 
-// Row r of the 32B-swizzled readout operand (see store_state_row_sw32) from 40 bf16 pairs.
+// Row r of the 32B-swizzled readout operand (see store_state_row_sw32) from NVC / 2 bf16
+// pairs (one 16-column atom per 8 pairs).
+template <int NVC>
 __device__ __forceinline__ void restage_store(uint32_t sbf, int r, const uint32_t* pk) {
   const uint32_t rb = sbf + (r >> 3) * 256 + (r & 7) * 32;
   const uint32_t flip = (r >> 2) & 1;
 #pragma unroll
-  for (int a = 0; a < 5; ++a)
+  for (int a = 0; a < NVC / 16; ++a)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const uint32_t* x = pk + a * 8 + hh * 4;
@@ -130,6 +139,7 @@ __device__ __forceinline__ float corners_h5(const Corners& k, int g) {
          ((g & 4) ? k.f7[1] : k.f7[0]);
 }
 
+template <int NVC>
 __global__ void __launch_bounds__(kSPThreads, 1)
     k_sweep_pipe(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, const float* __restrict__ W,
@@ -254,8 +264,8 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     // half starts once that half of the state after chunk c has been read out.
     const uint32_t id_proj = idesc_bf16(128, 16, 0, 0);
     const uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
-    const uint32_t id_ro = idesc_bf16(128, kNV, 0, 1);   // A tmem (K-major), B MN-major
-    const uint32_t id_up = idesc_bf16(128, kNV, 1, 1);   // A MN-major smem, B MN-major
+    const uint32_t id_ro = idesc_bf16(128, NVC, 0, 1);   // A tmem (K-major), B MN-major
+    const uint32_t id_up = idesc_bf16(128, NVC, 1, 1);   // A MN-major smem, B MN-major
     // Start addresses stay below 2^18 bytes, so adding (bytes >> 4) to a descriptor
     // never carries out of its 14-bit field.
     const uint64_t d_w = sdesc(sb + SPSmem::w, 128, 1024, kSwizzleNone);
@@ -559,13 +569,13 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       for (int hf = 0; hf < 2; ++hf) {
         if (!wait(sp_UPD0 + hf, par)) break;
         tc_fence_after();
-        uint32_t pk[40];
-        restage_load(tmem + lane_off + (hf ? SPTm::S1 : SPTm::S0), pk);
+        uint32_t pk[NVC / 2];
+        restage_load<NVC>(tmem + lane_off + (hf ? SPTm::S1 : SPTm::S0), pk);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar + sp_SREAD0 + hf);
         if (hf == 0 && !wait(sp_PQ_FREE, par)) break;   // RO(x) read the state of chunk x-1
-        restage_store(sb + SPSmem::sbf, 128 * hf + t, pk);
+        restage_store<NVC>(sb + SPSmem::sbf, 128 * hf + t, pk);
         if (t == 0) SW_TRACE(x, 32 + hf);
       }
       if (!ok) break;
@@ -597,7 +607,8 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       uint32_t acc[72];
 #pragma unroll
       for (int b = 0; b < 4; ++b) tmem_ld16(tmem + lane_off + SPTm::num + b * 16, acc + b * 16);
-      tmem_ld8(tmem + lane_off + SPTm::num + 64, acc + 64);
+      if (NVC == 80) tmem_ld8(tmem + lane_off + SPTm::num + 64, acc + 64);
+      else acc[64] = 0u;   // no denominator column: the dv pass reads the numerator only
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
