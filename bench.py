@@ -384,7 +384,10 @@ def run_ours(args, wl: I.Workload):
         "clocks": clocks,
     }
     if not args.no_e2e:
-        line["e2e"] = run_e2e(args, wl, x, a, ra, dev, stream, world, backward)
+        outs = {"out": out}
+        if backward:
+            outs.update(dq=dq, dk=dk, dv=dv, dW=dW)
+        line["e2e"] = run_e2e(args, wl, x, outs, a, ra, dev, stream, world, backward)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n = args.cpu_tokens
         rate, dt, cores = oracle_rate(wl, n, backward)
@@ -399,110 +402,82 @@ def run_ours(args, wl: I.Workload):
         dist.destroy_process_group()
 
 
-def run_e2e(args, wl, x, a, ra, dev, stream, world, backward):
+def run_e2e(args, wl, x, outs, a, ra, dev, stream, world, backward):
     """Same step through the public API with host inputs: pinned host -> device copies
-    of q, k, v (and dO), the step, device -> host copies of the results.
+    of q, k, v (and dO), the step, device -> host copies of the results (o, and dq, dk,
+    dv, dW for the backward), every step.
 
-    The heads go in two groups (when the head count is even): the inputs of group 2
-    upload while group 1 computes, and the results of group 1 download while group 2
-    computes, on two copy streams (one cudaMemcpyAsync per tensor slice).  With 4 of 8
-    heads per call the sweeps still fill one wave of CTAs, so the grouping costs the
-    kernels nothing; dW of the shared planes is the sum of the groups' dW."""
+    Steps alternate between two device buffer sets (set 0 is the device-timed run's own
+    tensors `x` and `outs`, set 1 is allocated here), so the inputs of step s + 1 upload
+    on one copy stream while step s computes, and the results of step s - 1 download on
+    another meanwhile (one cudaMemcpyAsync per tensor).  Every step computes all heads at
+    once, which keeps the sweeps' grids as wide as in the device-timed run.  The timed
+    region opens before the first upload and closes after the last download."""
     try:
         import torch.distributed as dist
         names = ["q", "k", "v"] + (["dout"] if backward else [])
-        H = x["q"].shape[0]
-        ng = 2 if H % 2 == 0 and H >= 2 else 1
-        hg = H // ng
+        res = ["out"] + (["dq", "dk", "dv", "dW"] if backward else [])
         host = {n: torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True) for n in names}
         for n in names:
             host[n].copy_(x[n])
-        dev_in = {n: torch.empty_like(x[n]) for n in names}
-        W = x["W"]
-        out = torch.empty_like(x["q"])
-        den = torch.empty(x["q"].shape[:2], dtype=torch.float32, device=dev)
-        per_head = [out]
-        if backward:
-            dq, dk, dv = (torch.empty_like(x[n]) for n in ("q", "k", "v"))
-            per_head += [dq, dk, dv]
-            dWg = [torch.empty_like(W) for _ in range(ng)]
-            dW = torch.empty_like(W)
-        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in per_head]
-        host_dW = torch.empty(W.shape, dtype=W.dtype, pin_memory=True) if backward else None
+        ins = [{n: x[n] for n in names}, {n: torch.empty_like(x[n]) for n in names}]
+        res_sets = [{n: outs[n] for n in res}, {n: torch.empty_like(outs[n]) for n in res}]
+        host_res = {n: torch.empty(outs[n].shape, dtype=outs[n].dtype, pin_memory=True)
+                    for n in res}
         h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-        d2h = sum(t.numel() * t.element_size() for t in per_head)
-        if backward:
-            d2h += W.numel() * W.element_size()
-        sl = [slice(g * hg, (g + 1) * hg) for g in range(ng)]
-        ga = []
-        for g in range(ng):
-            ag = ra.make_args(x["q"][sl[g]], W, wl.tau, wl.causal, chunk=wl.chunk,
-                              impl=args.kernels, den=den[sl[g]])
-            ag.workspace, ag.workspace_bytes = a.workspace, a.workspace_bytes
-            ga.append(ag)
+        d2h = sum(host_res[n].numel() * host_res[n].element_size() for n in res)
+        W = x["W"]
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev = lambda: torch.cuda.Event()  # noqa: E731
-        state = {"computed": [None] * ng, "downloaded": [None] * ng}
+        computed, downloaded = [None, None], [None, None]
 
-        def step():
-            uploaded = []
-            for g in range(ng):
-                with torch.cuda.stream(up):
-                    if state["computed"][g] is not None:   # last step's compute read them
-                        up.wait_event(state["computed"][g])
-                    for n in names:
-                        dev_in[n][sl[g]].copy_(host[n][sl[g]], non_blocking=True)
-                    e = ev()
-                    e.record(up)
-                    uploaded.append(e)
-            for g in range(ng):
-                stream.wait_event(uploaded[g])
-                if state["downloaded"][g] is not None:   # last step's results were read
-                    stream.wait_event(state["downloaded"][g])
-                d = {n: dev_in[n][sl[g]] for n in names}
-                ra.race_forward_ex(d["q"], d["k"], d["v"], W, out[sl[g]], ga[g], stream)
-                if backward:
-                    ra.race_backward_ex(d["q"], d["k"], d["v"], W, out[sl[g]], d["dout"],
-                                        dq[sl[g]], dk[sl[g]], dv[sl[g]], dWg[g], ga[g], stream)
-                e = ev()
-                e.record(stream)
-                state["computed"][g] = e
-                with torch.cuda.stream(down):
-                    down.wait_event(e)
-                    for t, hst in zip(per_head, host_out):
-                        hst[sl[g]].copy_(t[sl[g]], non_blocking=True)
-                    e2 = ev()
-                    e2.record(down)
-                    state["downloaded"][g] = e2
+        def step(s):
+            b = s & 1
+            d, r = ins[b], res_sets[b]
+            with torch.cuda.stream(up):
+                if computed[b] is not None:     # step s - 2 has read this input set
+                    up.wait_event(computed[b])
+                for n in names:
+                    d[n].copy_(host[n], non_blocking=True)
+                uploaded = torch.cuda.Event()
+                uploaded.record(up)
+            stream.wait_event(uploaded)
+            if downloaded[b] is not None:       # step s - 2's results have left this set
+                stream.wait_event(downloaded[b])
+            ra.race_forward_ex(d["q"], d["k"], d["v"], W, r["out"], a, stream)
             if backward:
-                torch.sum(torch.stack(dWg), dim=0, out=dW)
-                allreduce_dw(dW, world)
-                e = ev()
-                e.record(stream)
-                with torch.cuda.stream(down):
-                    down.wait_event(e)
-                    host_dW.copy_(dW, non_blocking=True)
-            end = ev()
-            end.record(down)
-            stream.wait_event(end)
+                ra.race_backward_ex(d["q"], d["k"], d["v"], W, r["out"], d["dout"],
+                                    r["dq"], r["dk"], r["dv"], r["dW"], a, stream)
+                allreduce_dw(r["dW"], world)
+            computed[b] = torch.cuda.Event()
+            computed[b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                for n in res:
+                    host_res[n].copy_(r[n], non_blocking=True)
+                downloaded[b] = torch.cuda.Event()
+                downloaded[b].record(down)
+            return downloaded[b]
 
-        n = max(1, min(args.steps, args.e2e_steps))
-        step()
+        n = max(1, min(args.steps, args.e2e_steps) if args.e2e_steps > 0 else args.steps)
+        for s in range(2):                      # warm-up: both buffer sets once
+            step(s)
+        torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        torch.cuda.synchronize(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(n):
-            step()
+        up.wait_event(e0)
+        for s in range(n):
+            last = step(s)
+        stream.wait_event(last)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
         tokens = wl.batch * wl.N * world
         return {"value": tokens / (ms / 1000), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": ms, "steps": n, "head_groups": ng}
+                "ms_per_step": ms, "steps": n, "buffer_sets": 2}
     except Exception as e:  # pinned host memory can be short on some hosts
         return {"value": None, "unit": "tokens/s", "error": repr(e)[:200]}
 
@@ -518,7 +493,8 @@ def main():
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--kernels", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="steps of the end-to-end leg (0: the same as --steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=8192)
     ap.add_argument("--ref-tokens", type=int, default=2048)
