@@ -428,35 +428,55 @@ def run_e2e(args, wl, x, outs, a, ra, dev, stream, world, backward):
         d2h = sum(host_res[n].numel() * host_res[n].element_size() for n in res)
         W = x["W"]
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        computed, downloaded = [None, None], [None, None]
+        fwd_in = [n for n in names if n != "dout"]
+        grads = [n for n in res if n != "out"]
+        # per buffer set: compute done reading its inputs; its o and its gradients copied out
+        computed, out_read, grads_read = [None, None], [None, None], [None, None]
+
+        def event(st):
+            e = torch.cuda.Event()
+            e.record(st)
+            return e
 
         def step(s):
+            # The forward needs q, k, v only and o is final after it: the forward starts
+            # before dO has landed, and o downloads while the backward runs.
             b = s & 1
             d, r = ins[b], res_sets[b]
             with torch.cuda.stream(up):
                 if computed[b] is not None:     # step s - 2 has read this input set
                     up.wait_event(computed[b])
-                for n in names:
+                for n in fwd_in:
                     d[n].copy_(host[n], non_blocking=True)
-                uploaded = torch.cuda.Event()
-                uploaded.record(up)
-            stream.wait_event(uploaded)
-            if downloaded[b] is not None:       # step s - 2's results have left this set
-                stream.wait_event(downloaded[b])
+                fwd_ready = event(up)
+                if backward:
+                    d["dout"].copy_(host["dout"], non_blocking=True)
+                    bwd_ready = event(up)
+            stream.wait_event(fwd_ready)
+            if out_read[b] is not None:         # step s - 2's o has left this set
+                stream.wait_event(out_read[b])
             ra.race_forward_ex(d["q"], d["k"], d["v"], W, r["out"], a, stream)
+            fwd_done = event(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(fwd_done)
+                host_res["out"].copy_(r["out"], non_blocking=True)
+                out_read[b] = event(down)
             if backward:
+                stream.wait_event(bwd_ready)
+                if grads_read[b] is not None:   # step s - 2's gradients have left this set
+                    stream.wait_event(grads_read[b])
                 ra.race_backward_ex(d["q"], d["k"], d["v"], W, r["out"], d["dout"],
                                     r["dq"], r["dk"], r["dv"], r["dW"], a, stream)
                 allreduce_dw(r["dW"], world)
-            computed[b] = torch.cuda.Event()
-            computed[b].record(stream)
+            computed[b] = event(stream)
+            if not backward:
+                return out_read[b]
             with torch.cuda.stream(down):
                 down.wait_event(computed[b])
-                for n in res:
+                for n in grads:
                     host_res[n].copy_(r[n], non_blocking=True)
-                downloaded[b] = torch.cuda.Event()
-                downloaded[b].record(down)
-            return downloaded[b]
+                grads_read[b] = event(down)
+            return grads_read[b]
 
         n = max(1, min(args.steps, args.e2e_steps) if args.e2e_steps > 0 else args.steps)
         for s in range(2):                      # warm-up: both buffer sets once
