@@ -92,12 +92,13 @@ def kernel_work(name: str, wl: I.Workload):
 
 # DRAM bytes (read + write) per token-head of a launch, from one ncu capture of a smaller
 # launch of the same kernel and configuration (8 heads, N = 131,072, L = 16, P = 8,
-# `dram__bytes_read.sum + dram__bytes_write.sum`): 946 MB for the forward sweep (the
-# instantiation with the mass column; the dv pass's 64-column one reads and writes the
-# same arrays), 1,975 MB for the q side and 1,974 MB for the k side of the pipelined
+# `dram__bytes_read.sum + dram__bytes_write.sum`): 946 MB per launch of the causal sweep
+# (the mean of the forward's 80-column instantiation, 944 MB, and the dv pass's 64-column
+# one, 948 MB: the bench's per-launch time of the sweep is the mean of the same two
+# launches), 1,975 MB for the q side and 1,974 MB for the k side of the pipelined
 # backward sweep.  The traffic grows in proportion to H x N.
 DRAM_BYTES_PER_TOKEN_HEAD = {
-    "tc_causal_sweep": 946.05e6 / (8 * 131072),
+    "tc_causal_sweep": (698.695e6 + 247.275e6) / (8 * 131072),
     "tc_bwd_q": (1442.38e6 + 532.65e6) / (8 * 131072),
     "tc_bwd_k": (1442.33e6 + 531.99e6) / (8 * 131072),
 }
